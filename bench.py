@@ -1,0 +1,396 @@
+"""Benchmark of the DSA hot path: query tokens/s through indexer + top-k + sparse MLA.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path (dsa_forward: Lightning-Indexer
+scores, per-query top-k, sparse MLA) over one batch of synthetic inputs that
+already sit in HBM.  The default workload is the 32K-context chunked prefill
+(4096 new queries after a 28672-token prefix, top-2048, 128 MLA heads).
+Rank 0 prints one JSON line.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the workload (weak scaling, no data-path collective); value = all ranks'
+tokens / the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "query tokens/s through indexer+top-k+sparse MLA @32K ctx; % of roofline"
+UNIT = "query tokens/s"
+DEFAULT_WORKLOAD = "chunked_prefill_28k_4k"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------- work model
+def work_model(x):
+    """Algorithmic FLOPs and bytes of each stage for a DSAInputs batch."""
+    b = x.batch
+    t = b.q_pos.astype(np.int64)
+    n_valid = t + 1
+    pairs = int(n_valid.sum())
+    k = x.k_sel
+    n_sel = np.minimum(n_valid, k)
+    H = x.n_heads
+    # keys each sequence's queries can reach (max t + 1 per sequence)
+    reach = np.zeros(b.num_seqs, np.int64)
+    np.maximum.at(reach, b.q_seq, n_valid)
+    idx_flops = pairs * 2 * 64 * 128
+    idx_bytes = int(reach.sum()) * (128 + 4) + b.total_q * (64 * 128 + 64 * 4 * 2) + pairs * 4
+    topk_bytes = pairs * 4 + b.total_q * k * 4
+    mla_flops = int((n_sel * H).sum()) * 2 * (576 + 512)
+    # every latent row a sequence's selections may touch is read once (upper bound: the reachable prefix)
+    mla_bytes = int(np.minimum(reach, n_sel.max() * np.bincount(b.q_seq, minlength=b.num_seqs)).sum()) * 1152 \
+        + b.total_q * (H * 576 * 2 + H * 512 * 2 + k * 4 + H * 4)
+    return {"indexer": {"flops": idx_flops, "bytes": idx_bytes, "peak": "fp8"},
+            "topk": {"flops": 0, "bytes": topk_bytes, "peak": None},
+            "sparse_mla": {"flops": mla_flops, "bytes": mla_bytes, "peak": "bf16"}}
+
+
+def roofline_entry(stage, work, sec, pk, sustained=True):
+    tf = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    tensor_peak = {"fp8": 2.0 * tf, "bf16": tf, None: None}[work["peak"]]
+    t_flops = work["flops"] / (tensor_peak * 1e12) if tensor_peak else 0.0
+    t_bytes = work["bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_flops >= t_bytes:
+        achieved = work["flops"] / sec / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "ideal_us": t_flops * 1e6, "us": sec * 1e6}
+    achieved = work["bytes"] / sec / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "ideal_us": t_bytes * 1e6, "us": sec * 1e6}
+
+
+def ncu_traffic(kernel_file, kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source
+    is unchanged since the capture; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel_key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "long_context_sparse_lightning_b200", "csrc", kernel_file)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d.get("bytes_per_launch") if d.get("source_sha") == sha else None
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [v.strip() for v in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_rows_per_sec(x, budget_s=15.0, min_rows=4, max_rows=4096, seed=7):
+    """Time the fp64 oracle (scores -> top-k -> sparse MLA) on query rows of x
+    until ~budget_s of CPU time; returns (rows/s, rows done, seconds)."""
+    from oracle import indexer, mla, topk
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(x.batch.total_q)
+    done = 0
+    t0 = time.perf_counter()
+    while done < min(max_rows, x.batch.total_q):
+        r = int(order[done])
+        (_, t, I, B), = indexer.scores(x, [r])
+        sel, _ = topk.select(I, x.k_sel)
+        mla.sparse(x, topk.padded(sel, x.k_sel)[None, :], [r])
+        done += 1
+        el = time.perf_counter() - t0
+        if done >= min_rows and el >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# --------------------------------------------------------------------- main
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from dsa_inputs import make_inputs
+    x = make_inputs(args.workload, seed=0)
+    per_step = max(1, args.ref_rows)
+    times = []
+    done_rows = 0
+    for s in range(args.warmup + args.steps):
+        rps, n, el = oracle_rows_per_sec(x, budget_s=0.0, min_rows=per_step, max_rows=per_step, seed=100 + s)
+        if s >= args.warmup:
+            times.append(el)
+            done_rows += n
+    total = sum(times)
+    value = done_rows / total
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(x, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} query rows of {args.workload} per step (scores over the "
+                                       f"full causal prefix, exact top-k, sparse MLA), fp64 numpy"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(x, args):
+    b = x.batch
+    return {"workload": x.workload.name, "description": x.workload.description, "n_q": b.total_q,
+            "num_seqs": b.num_seqs, "max_kv_len": b.max_kv_len, "k_sel": x.k_sel, "n_heads": x.n_heads,
+            "index_heads": 64, "index_dim": 128, "latent_dim": 576, "value_dim": 512,
+            "l2": "flushed between timed steps (256 MiB write, outside the events)", "seed": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference step")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import long_context_sparse_lightning_b200 as dsa
+    from dsa_inputs import make_inputs
+    from dsa_inputs.torch_io import host_tensors
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = td
+
+    x = make_inputs(args.workload, seed=rank)
+    b = x.batch
+    host = host_tensors(x, pin=True)
+    t = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    batch = dsa.Batch(t["cu_q"], t["kv_len"], t["kv_start"], b.total_q, b.max_q_per_seq, b.max_kv_len, b.total_keys)
+    k, H = x.k_sel, x.n_heads
+    idx = torch.empty((b.total_q, k), dtype=torch.int32, device=dev)
+    out = torch.empty((b.total_q, H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b.total_q, H), dtype=torch.float32, device=dev)
+    ws = dsa.workspace(dsa.OP_FORWARD, batch, k, H, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    def step():
+        dsa.forward(batch, t["q8"], t["q_scale"], t["w"], t["k8"], t["k_scale"], k, t["q_mla"], t["latent"],
+                    x.sm_scale, idx, out, lse, ws)
+
+    for _ in range(args.warmup):
+        step()
+    dsa.check_device_error(ws)
+
+    # ---- headline: K steps on resident inputs, L2 flushed between steps ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    dsa.check_device_error(ws)
+    sec = sum(a.elapsed_time(c) for a, c in ev) / 1e3
+    if pg:
+        tt = torch.tensor([sec], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        sec = float(tt.item())
+    value = world * b.total_q * args.steps / sec
+    launches_per_step = 3 + (1 if dsa_nsplit(b, k) > 1 else 0)
+
+    # ---- per-stage device time (same stream, CUDA events between the launches) ----
+    ld = ((b.max_kv_len + 3) // 4) * 4
+    scores = torch.empty((b.total_q, ld), dtype=torch.float32, device=dev)
+    ws_s = dsa.workspace(dsa.OP_SPARSE_MLA, batch, k, H, device=dev)
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.fill_(float(i))
+        e = st_ev[i - args.warmup] if i >= args.warmup else None
+        if e: e[0].record(stream)
+        dsa.indexer_scores(batch, t["q8"], t["q_scale"], t["w"], t["k8"], t["k_scale"], scores, ws_s)
+        if e: e[1].record(stream)
+        dsa.topk(batch, scores, k, idx, ws_s)
+        if e: e[2].record(stream)
+        dsa.sparse_mla(batch, t["q_mla"], t["latent"], idx, k, x.sm_scale, out, lse, ws_s)
+        if e: e[3].record(stream)
+    torch.cuda.synchronize()
+    dsa.check_device_error(ws_s)
+    stage_sec = {name: sum(e[j].elapsed_time(e[j + 1]) for e in st_ev) / 1e3 / args.steps
+                 for j, name in enumerate(["indexer", "topk", "sparse_mla"])}
+    del scores
+
+    # ---- end to end through the C ABI from pinned host buffers ----
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in (out_h, idx_h, lse_h))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        e = e2e_ev[i - args.warmup] if i >= args.warmup else None
+        if e: e[0].record(stream)
+        for name, v in host.items():
+            t[name].copy_(v, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        idx_h.copy_(idx, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        if e: e[1].record(stream)
+        torch.cuda.synchronize()
+    e2e_sec = sum(a.elapsed_time(c) for a, c in e2e_ev) / 1e3
+    if pg:
+        tt = torch.tensor([e2e_sec], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e2e_sec = float(tt.item())
+    e2e_value = world * b.total_q * args.steps / e2e_sec
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    pk = peaks()
+    wm = work_model(x)
+    stages = {n: roofline_entry(n, wm[n], stage_sec[n], pk) for n in stage_sec}
+    dom = max(stage_sec, key=stage_sec.get)
+    kfile = {"indexer": "indexer_sm100.cu", "topk": "topk.cu", "sparse_mla": "sparse_mla_sm100.cu"}[dom]
+    roof = dict(stages[dom])
+    roof["kernel"] = dom
+    roof["traffic"] = ncu_traffic(kfile, dom)
+    roof["peak_source"] = pk["source"] + (" sustained" if roof["unit"] == "TFLOP/s" else "")
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        rps, n_rows, el = oracle_rows_per_sec(x, budget_s=args.cpu_budget)
+        cpu = {"value": rps, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{n_rows} query rows of {args.workload} ({el:.1f} s): fp64 scores over each row's "
+                         f"causal prefix, exact top-k, sparse MLA"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+f16", "data": "synthetic",
+            "config": config_of(x, args), "roofline": roof,
+            "stages": {n: {k2: v for k2, v in s.items()} for n, s in stages.items()},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def dsa_nsplit(b, k_sel):
+    # mirrors the library's split heuristic for the launch count (>= 4 tiles per split, fill 148 SMs)
+    tiles = (k_sel + 63) // 64
+    s = 1
+    while s * 2 <= tiles // 4 and b.total_q * s < 148:
+        s *= 2
+    return s
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,163 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * Three stages, each one hand-written CUDA kernel, plus their composition:
+ *
+ *   dsa_indexer_scores  Lightning-Indexer scores, Eq. (1) of "详解DSA":
+ *                         I[t,s] = sum_{j<64} w[t,j] * ReLU(q[t,j] . k[s]),  s <= t,
+ *                       on FP8 e4m3 q and k with one fp32 scale per 128-element
+ *                       vector (the demo Indexer.forward of "详解DSA" quantises q
+ *                       and k per 128 and hands codes + scales to its FP8 index
+ *                       kernel).  The scales are folded exactly:
+ *                         I = k_scale[s] * sum_j (w*q_scale)[t,j] * ReLU(q8[t,j] . k8[s]).
+ *   dsa_topk            per query row, the k_sel positions of largest score among
+ *                       s <= t, Eq. (2) of "详解DSA" (S_t = {s : I[t,s] in Top-k});
+ *                       rows with at most k_sel positions keep all of them (the
+ *                       demo takes topk(min(index_topk, end_pos))).
+ *   dsa_sparse_mla      attention of all n_heads query heads of a token over the
+ *                       selected latent entries, MQA mode ("DeepSeek V3.2
+ *                       稀疏注意力", section on embedding DSA in MLA: every head of
+ *                       a token shares the same top-k latent KV entries):
+ *                         o[h] = sum_i softmax_i(sm_scale * q[h] . c[s_i]) * c[s_i][0:512]
+ *                       over 576-d entries (512 latent + 64 RoPE), value = first 512.
+ *   dsa_forward         indexer -> top-k -> sparse MLA on one stream
+ *                       (T_DSA = T_index + T_topk + T_gather + T_sparse_attn,
+ *                       "DeepSeek V3.2 稀疏注意力", complexity section).
+ *
+ * Conventions (all entry points):
+ *   - Every tensor pointer is caller-owned DEVICE memory, row-major and
+ *     contiguous, 16-byte aligned.  The library never allocates, never frees
+ *     and keeps no per-call global state.
+ *   - Every call is asynchronous on `stream` and never synchronises, except
+ *     dsa_check_device_error.  Argument errors are returned before any launch.
+ *   - Positions (indices) are sequence-relative int32, as torch.topk returns
+ *     positions in the demo; a selection is a set: valid entries first, then -1.
+ *   - Unsupported shapes return DSA_ERR_UNSUPPORTED; there is no fallback path.
+ *   - `ws` is a caller-provided device workspace of at least
+ *     dsa_workspace_size(op, ...) bytes.  Its first 16 bytes are a device error
+ *     word that kernels set when a bounded wait times out or an index is out of
+ *     range; zero the workspace once after allocating it, and read (and clear)
+ *     the word with dsa_check_device_error.
+ *
+ * Ragged batches: query row r belongs to sequence b with cu_q[b] <= r < cu_q[b+1];
+ * its i-th query (i = r - cu_q[b]) sits at position t = kv_len[b] - q_len[b] + i,
+ * q_len[b] = cu_q[b+1] - cu_q[b], and may see positions 0..t.  Key/latent row of
+ * position s of sequence b is kv_start[b] + s in the flat caches.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL = the legacy default stream. */
+typedef struct CUstream_st* dsa_stream_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer          */
+  DSA_ERR_UNSUPPORTED = 2,     /* a shape the kernels do not implement                */
+  DSA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed                   */
+  DSA_ERR_WORKSPACE = 4,       /* ws too small                                        */
+  DSA_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (device error word) */
+  DSA_ERR_DEVICE_BOUNDS = 6    /* a kernel met an out-of-range index (device word)    */
+} dsa_status_t;
+
+typedef enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MLA = 2,
+  DSA_OP_FORWARD = 3
+} dsa_op_t;
+
+/* Host struct describing a ragged batch; the three arrays are DEVICE memory. */
+typedef struct {
+  int32_t num_seqs;          /* B >= 1                                             */
+  int32_t total_q;           /* cu_q[B]; query rows of every per-row tensor       */
+  int32_t max_q_per_seq;     /* max_b q_len[b] (host copy, sizes the grids)       */
+  int32_t max_kv_len;        /* max_b kv_len[b] (host copy)                       */
+  int64_t total_keys;        /* rows of the flat key / latent caches (< 2^31)     */
+  const int32_t* cu_q;       /* [B+1] query-row offsets, cu_q[0] = 0              */
+  const int32_t* kv_len;     /* [B] positions present, including the new queries  */
+  const int64_t* kv_start;   /* [B] first flat cache row of each sequence          */
+} dsa_batch_t;
+
+/* Fixed sizes of the hot path (the pages' indexer: 64 heads of dim 128). */
+#define DSA_INDEX_HEADS 64
+#define DSA_INDEX_DIM 128
+#define DSA_LATENT_DIM 576
+#define DSA_VALUE_DIM 512
+#define DSA_MAX_K_SEL 2048
+
+/* Bytes of device workspace the call `op` needs for this batch.  Returns 0
+ * when the arguments are invalid.  For DSA_OP_FORWARD this includes the
+ * [total_q, ld] fp32 score matrix, ld = max_kv_len rounded up to 4. */
+DSA_API size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads);
+
+/* Indexer scores.
+ *   q_fp8   [total_q, 64, 128] e4m3 codes      q_scale [total_q, 64] fp32 (> 0)
+ *   w       [total_q, 64] fp32                 k_fp8   [total_keys, 128] e4m3 codes
+ *   k_scale [total_keys] fp32 (> 0)
+ *   scores  [total_q, ld_scores] fp32 out; row r holds I[t, s] for s = 0..t of its
+ *           sequence; entries beyond t are not written.  ld_scores >= max_kv_len,
+ *           a multiple of 4. */
+DSA_API dsa_status_t dsa_indexer_scores(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale,
+                                const float* w, const void* k_fp8, const float* k_scale, float* scores,
+                                int64_t ld_scores, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Top-k positions per query row.
+ *   scores [total_q, ld_scores] fp32 (only s <= t is read)
+ *   idx    [total_q, k_sel] int32 out: the selected positions (ties: lower s
+ *          first), then -1 padding when t + 1 < k_sel.
+ *   1 <= k_sel <= 2048. */
+DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int64_t ld_scores, int32_t k_sel,
+                      int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Sparse MLA (MQA mode).
+ *   q    [total_q, n_heads, 576] bf16        kv [total_keys, 576] bf16 latent cache
+ *   idx  [total_q, k_sel] int32 positions; entries < 0 or >= kv_len are skipped
+ *   out  [total_q, n_heads, 512] bf16 (round to nearest even from fp32)
+ *   lse  [total_q, n_heads] fp32 natural-log sum-exp of the scaled logits, or NULL.
+ *   A row with no usable entry gives out = 0, lse = -inf.
+ *   1 <= n_heads <= 128 (one 128-row MMA tile; fewer heads leave rows idle);
+ *   k_sel as for dsa_topk.  Internally q and the gathered entries are
+ *   converted to fp16 (exact for |x| in [2^-14, 65504]; larger magnitudes
+ *   saturate) and the softmax probabilities are rounded to fp16. */
+DSA_API dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
+                            const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
+                            size_t ws_bytes, dsa_stream_t stream);
+
+/* The whole hot path: indexer scores (kept in ws), top-k into `idx`, sparse
+ * MLA into `out`/`lse`.  Arguments as above. */
+DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale, const float* w,
+                         const void* k_fp8, const float* k_scale, int32_t k_sel, const void* q, int32_t n_heads,
+                         const void* kv, float sm_scale, int32_t* idx, void* out, float* lse, void* ws,
+                         size_t ws_bytes, dsa_stream_t stream);
+
+/* Synchronise `stream`, read the device error word of `ws`, clear it, and
+ * return DSA_OK, DSA_ERR_DEVICE_TIMEOUT or DSA_ERR_DEVICE_BOUNDS (or
+ * DSA_ERR_CUDA if the stream reports an error).  `site` / `info`, if not NULL,
+ * receive the kernel site id and detail recorded with the error. */
+DSA_API dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info);
+
+/* Static description of a status code. */
+DSA_API const char* dsa_status_string(dsa_status_t status);
+
+/* ABI version (major * 100 + minor). */
+DSA_API int32_t dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,333 @@
+// C ABI of the DSA hot path: argument validation, workspace carving, TMA
+// descriptor encoding and kernel launches.  No allocation, no synchronisation
+// (except dsa_check_device_error), no fallback path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "kernels.cuh"
+
+namespace {
+
+using dsa::IndexerParams;
+using dsa::MlaParams;
+using dsa::TopkParams;
+
+constexpr size_t kHeaderBytes = 256;      // device error word + reserved
+constexpr long long kDefaultBudget = 2000000000LL;   // clock64 cycles per bounded wait (~1 s)
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long wait_budget() {
+  const char* s = std::getenv("DSA_WAIT_BUDGET_CYCLES");
+  if (s != nullptr) {
+    const long long v = std::atoll(s);
+    if (v > 0) return v;
+  }
+  return kDefaultBudget;
+}
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point ----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols].
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, size_t elem, uint64_t rows,
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+dsa_status_t check_batch(const dsa_batch_t* b) {
+  if (b == nullptr) return DSA_ERR_INVALID_ARG;
+  if (b->num_seqs < 1 || b->num_seqs > 65535 || b->total_q < 0 || b->max_q_per_seq < 0 || b->max_kv_len < 0 ||
+      b->total_keys < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (b->cu_q == nullptr || b->kv_len == nullptr || b->kv_start == nullptr) return DSA_ERR_INVALID_ARG;
+  if (b->total_q > 0 && (b->max_q_per_seq < 1 || b->max_kv_len < b->max_q_per_seq || b->total_keys < 1))
+    return DSA_ERR_INVALID_ARG;
+  if (b->max_q_per_seq > b->total_q || static_cast<int64_t>(b->max_kv_len) > b->total_keys)
+    return DSA_ERR_INVALID_ARG;
+  if (b->total_keys >= (int64_t(1) << 31) || static_cast<int64_t>(b->total_q) * 128 >= (int64_t(1) << 31))
+    return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < need) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+int64_t forward_ld(const dsa_batch_t* b) { return static_cast<int64_t>(align_up(b->max_kv_len, 4)); }
+
+struct MlaSplit {
+  int nsplit;
+  int keys_per_split;
+};
+MlaSplit mla_split(const dsa_batch_t* b, int k_sel) {
+  const int s = dsa::mla_num_splits(b->total_q, b->max_q_per_seq, b->num_seqs, k_sel);
+  return {s, dsa::mla_keys_per_split(k_sel, s)};
+}
+
+size_t mla_part_bytes(const dsa_batch_t* b, int k_sel) {
+  const MlaSplit sp = mla_split(b, k_sel);
+  if (sp.nsplit <= 1) return 0;
+  const size_t rows = static_cast<size_t>(b->total_q) * sp.nsplit * 128;
+  return align_up(rows * 512 * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
+}
+
+// ----------------------------------------------------------------- stages --
+dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q_scale, const float* w,
+                         const void* k_fp8, const float* k_scale, float* scores, int64_t ld, uint32_t* err,
+                         cudaStream_t stream) {
+  const int tok = dsa::indexer_tokens_per_cta(b->max_q_per_seq);
+  CUtensorMap tq, tk;
+  if (!make_tmap_2d(&tq, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_q) * 64, 128,
+                    dsa::indexer_box_rows_q(tok), 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128, 128,
+                    128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  const int qblocks = (b->max_q_per_seq + tok - 1) / tok;
+  if (qblocks > 65535) return DSA_ERR_UNSUPPORTED;
+  const int tiles = (b->max_kv_len + 127) / 128;
+  const int64_t target = int64_t(8) * 148;   // one CTA per SM (registers), ~8 waves
+  int tpc = tiles;
+  while (tpc > 8 && static_cast<int64_t>(b->num_seqs) * qblocks * ((tiles + tpc - 1) / tpc) < target)
+    tpc = (tpc + 1) / 2;
+  IndexerParams p;
+  p.cu_q = b->cu_q;
+  p.kv_len = b->kv_len;
+  p.kv_start = b->kv_start;
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.scores = scores;
+  p.ld = ld;
+  p.total_keys = b->total_keys;
+  p.tiles_per_chunk = tpc;
+  p.num_qblocks = qblocks;
+  p.err = err;
+  p.budget = wait_budget();
+  const dim3 grid((tiles + tpc - 1) / tpc, qblocks, b->num_seqs);
+  return dsa::launch_indexer(tok, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int k_sel, int32_t* idx,
+                      uint32_t* err, cudaStream_t stream) {
+  TopkParams p;
+  p.cu_q = b->cu_q;
+  p.kv_len = b->kv_len;
+  p.scores = scores;
+  p.ld = ld;
+  p.k_sel = k_sel;
+  p.idx = idx;
+  p.err = err;
+  const dim3 grid(b->max_q_per_seq, b->num_seqs);
+  return dsa::launch_topk(b->max_kv_len, grid, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const void* kv, const int32_t* idx,
+                     int k_sel, float sm_scale, void* out, float* lse, uint8_t* part, uint32_t* err,
+                     cudaStream_t stream) {
+  const MlaSplit sp = mla_split(b, k_sel);
+  MlaParams p;
+  p.cu_q = b->cu_q;
+  p.kv_len = b->kv_len;
+  p.kv_start = b->kv_start;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = static_cast<const uint16_t*>(kv);
+  p.idx = idx;
+  p.total_keys = b->total_keys;
+  p.k_sel = k_sel;
+  p.n_heads = n_heads;
+  p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.nsplit = sp.nsplit;
+  p.keys_per_split = sp.keys_per_split;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  if (sp.nsplit > 1) {
+    const size_t rows = static_cast<size_t>(b->total_q) * sp.nsplit * 128;
+    p.part_o = reinterpret_cast<float*>(part);
+    p.part_lse = reinterpret_cast<float*>(part + align_up(rows * 512 * sizeof(float), 256));
+  }
+  p.err = err;
+  p.budget = wait_budget();
+  const int64_t gx = int64_t(2) * b->max_q_per_seq * sp.nsplit;
+  if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
+  if (dsa::launch_sparse_mla(grid, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (sp.nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status_t check_indexer_args(const dsa_batch_t* b, const void* q_fp8, const float* q_scale, const float* w,
+                                const void* k_fp8, const float* k_scale) {
+  if (q_fp8 == nullptr || q_scale == nullptr || w == nullptr || k_fp8 == nullptr || k_scale == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_fp8) || !aligned16(k_fp8) || !aligned16(q_scale) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  (void)b;
+  return DSA_OK;
+}
+
+dsa_status_t check_mla_args(const void* q, int n_heads, const void* kv, int k_sel, float sm_scale, void* out) {
+  if (q == nullptr || kv == nullptr || out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return DSA_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_heads > 128) return DSA_ERR_UNSUPPORTED;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads) {
+  if (check_batch(batch) != DSA_OK) return 0;
+  switch (op) {
+    case DSA_OP_INDEXER:
+    case DSA_OP_TOPK:
+      return kHeaderBytes;
+    case DSA_OP_SPARSE_MLA:
+      if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
+      return kHeaderBytes + mla_part_bytes(batch, k_sel);
+    case DSA_OP_FORWARD: {
+      if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
+      const size_t scores = align_up(static_cast<size_t>(batch->total_q) * forward_ld(batch) * sizeof(float), 256);
+      return kHeaderBytes + scores + mla_part_bytes(batch, k_sel);
+    }
+  }
+  return 0;
+}
+
+dsa_status_t dsa_indexer_scores(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale, const float* w,
+                                const void* k_fp8, const float* k_scale, float* scores, int64_t ld_scores, void* ws,
+                                size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer_args(batch, q_fp8, q_scale, w, k_fp8, k_scale)) != DSA_OK) return s;
+  if (scores == nullptr || !aligned16(scores) || ld_scores < batch->max_kv_len || (ld_scores & 3) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  return run_indexer(batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ld_scores, static_cast<uint32_t*>(ws),
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int64_t ld_scores, int32_t k_sel, int32_t* idx,
+                      void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if (scores == nullptr || idx == nullptr || !aligned16(scores) || ld_scores < batch->max_kv_len ||
+      (ld_scores & 3) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  return run_topk(batch, scores, ld_scores, k_sel, idx, static_cast<uint32_t*>(ws),
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
+                            const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
+                            size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_mla_args(q, n_heads, kv, k_sel, sm_scale, out)) != DSA_OK) return s;
+  if (idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes + mla_part_bytes(batch, k_sel))) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, static_cast<uint8_t*>(ws) + kHeaderBytes,
+                 static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale, const float* w,
+                         const void* k_fp8, const float* k_scale, int32_t k_sel, const void* q, int32_t n_heads,
+                         const void* kv, float sm_scale, int32_t* idx, void* out, float* lse, void* ws,
+                         size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer_args(batch, q_fp8, q_scale, w, k_fp8, k_scale)) != DSA_OK) return s;
+  if ((s = check_mla_args(q, n_heads, kv, k_sel, sm_scale, out)) != DSA_OK) return s;
+  if (idx == nullptr) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_workspace_size(DSA_OP_FORWARD, batch, k_sel, n_heads);
+  if ((s = check_ws(ws, ws_bytes, need)) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  const int64_t ld = forward_ld(batch);
+  float* scores = reinterpret_cast<float*>(base + kHeaderBytes);
+  uint8_t* part = base + kHeaderBytes + align_up(static_cast<size_t>(batch->total_q) * ld * sizeof(float), 256);
+  if ((s = run_indexer(batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ld, err, st)) != DSA_OK) return s;
+  if ((s = run_topk(batch, scores, ld, k_sel, idx, err, st)) != DSA_OK) return s;
+  return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, part, err, st);
+}
+
+dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info) {
+  if (ws == nullptr) return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t word[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (word[0] != 0) {
+    if (cudaMemset(ws, 0, sizeof(word)) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  if (site != nullptr) *site = word[1];
+  if (info != nullptr) *info = word[2];
+  switch (word[0]) {
+    case 0: return DSA_OK;
+    case DSA_ERR_DEVICE_TIMEOUT: return DSA_ERR_DEVICE_TIMEOUT;
+    case DSA_ERR_DEVICE_BOUNDS: return DSA_ERR_DEVICE_BOUNDS;
+    default: return DSA_ERR_CUDA;
+  }
+}
+
+const char* dsa_status_string(dsa_status_t status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_DEVICE_BOUNDS: return "device index out of range";
+  }
+  return "unknown status";
+}
+
+int32_t dsa_version(void) { return 100; }
+
+}  // extern "C"

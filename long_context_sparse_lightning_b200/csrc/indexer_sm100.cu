@@ -1,0 +1,301 @@
+// Lightning-Indexer scores on sm_100a: a tcgen05 FP8 contraction fed by TMA,
+// with ReLU, the w-weighted head sum and both FP8 scales fused into the
+// epilogue, so no [t, s, head] tensor ever exists.
+//
+//   I[t, s] = k_scale[s] * sum_j (w[t, j] * q_scale[t, j]) * ReLU(q8[t, j] . k8[s])
+//
+// which equals Eq. (1) of "详解DSA" on the dequantised q and k because the
+// scales are positive and ReLU is positively homogeneous ("详解DSA", prefill
+// analysis: the q scale multiplies w before the head sum, the k scale
+// multiplies the summed result).
+//
+// Tile mapping (one CTA = TOK query tokens of one sequence x a range of
+// 128-key tiles):
+//   MMA  M = 128 keys (TMEM lanes), N = tokens x 64 heads (TMEM columns),
+//        K = 128 FP8 dims = 4 x kind::f8f6f4 K32 instructions;
+//        A = k tile [128 x 128 B] and B = q tile [N x 128 B], both K-major,
+//        128-byte swizzled exactly as TMA writes them.
+//   Each epilogue thread owns one key (one TMEM lane) and reads that key's 64
+//   head values of a token from its own TMEM columns, so the head sum needs no
+//   cross-thread traffic; a warp stores 32 consecutive scores (128 B).
+//   Two accumulators in TMEM ping-pong between the MMA warp and two epilogue
+//   warpgroups (group g drains buffer g).
+//
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner),
+// warps 2..9 = epilogue (two warpgroups).
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+
+template <int TOK>
+struct IdxCfg {
+  static constexpr int NG = TOK == 8 ? 2 : 1;         // accumulator groups per key tile
+  static constexpr int GTOK = TOK / NG;               // tokens per group
+  static constexpr int N = GTOK * 64;                 // MMA N
+  static constexpr int STAGES = TOK >= 4 ? 6 : 8;
+  static constexpr int TMEM_COLS = 2 * N;             // 128, 256 or 512 (powers of two)
+  static constexpr int BOXQ = TOK * 64 < 256 ? TOK * 64 : 256;   // q rows per TMA box
+  static constexpr int Q_BYTES = TOK * 64 * 128;
+  static constexpr int K_BYTES = 128 * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_W = OFF_K + STAGES * K_BYTES;
+  static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 1 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-byte alignment
+  static_assert(OFF_K % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle-128 tiles need 1024-byte alignment");
+};
+
+template <int TOK>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                   const IndexerParams p) {
+  using C = IdxCfg<TOK>;
+  extern __shared__ uint8_t smem_raw[];
+
+  // ---- work unit: sequence b, query block, key-tile chunk ----
+  if (error_pending(p.err)) return;
+  const int b = blockIdx.z;
+  const int qblock = p.num_qblocks - 1 - static_cast<int>(blockIdx.y);   // long causal rows first
+  const int q0 = __ldg(&p.cu_q[b]);
+  const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
+  const int kv = __ldg(&p.kv_len[b]);
+  const int first = qblock * TOK;
+  if (first >= q_len) return;
+  const int64_t kstart = __ldg(&p.kv_start[b]);
+  if (q_len > kv || kv > p.ld || kstart < 0 || kstart + kv > p.total_keys) {
+    if (threadIdx.x == 0) report_error(p.err, kDevErrBounds, 101, b);
+    return;
+  }
+  const int ntok = min(TOK, q_len - first);
+  const int t_first = kv - q_len + first;
+  const int t_last = t_first + ntok - 1;
+  const int tiles_total = (t_last + 1 + 127) / 128;
+  const int tile_begin = static_cast<int>(blockIdx.x) * p.tiles_per_chunk;
+  if (tile_begin >= tiles_total) return;
+  const int n_tiles = min(tile_begin + p.tiles_per_chunk, tiles_total) - tile_begin;
+  const int row0 = q0 + first;
+
+  // ---- shared memory carve-up (1024-byte aligned base) ----
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = sm + C::OFF_Q;
+  uint8_t* sK = sm + C::OFF_K;
+  float* sW = reinterpret_cast<float*>(sm + C::OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* q_full = bars + 2 * C::STAGES;
+  uint64_t* acc_full = q_full + 1;    // [2]
+  uint64_t* acc_empty = q_full + 3;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  // w' = w * q_scale for this CTA's tokens (0 for rows past the sequence)
+  for (int i = threadIdx.x; i < TOK * 64; i += kThreads) {
+    const int tk = i >> 6;
+    float v = 0.f;
+    if (tk < ntok) {
+      const int64_t o = static_cast<int64_t>(row0 + tk) * 64 + (i & 63);
+      v = __ldg(&p.w[o]) * __ldg(&p.q_scale[o]);
+    }
+    sW[i] = v;
+  }
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);   // one arrival per epilogue warp of the group
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer --
+    if (elect_one()) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+      for (int piece = 0; piece < (TOK * 64) / C::BOXQ; ++piece) {
+        tma_load_2d(sQ + piece * C::BOXQ * 128, &tmap_q, q_full, 0, row0 * 64 + piece * C::BOXQ);
+      }
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 110, it);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], C::K_BYTES);
+        tma_load_2d(sK + s * C::K_BYTES, &tmap_k, &full[s], 0,
+                    static_cast<int32_t>(kstart + static_cast<int64_t>(tile_begin + it) * 128));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer --
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, C::N, 0, 0);
+      bool ok = mbar_wait(q_full, 0, p.budget);
+      if (!ok) report_error(p.err, kDevErrTimeout, 120, 0);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        if (!mbar_wait(&full[s], (it / C::STAGES) & 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 121, it);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sK + s * C::K_BYTES);
+#pragma unroll
+        for (int g = 0; g < C::NG; ++g) {
+          const int item = it * C::NG + g;
+          const int buf = item & 1;
+          if (!mbar_wait(&acc_empty[buf], ((item >> 1) & 1) ^ 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 122, it);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(sQ + g * C::N * 128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            umma_e4m3(tmem + buf * C::N, smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&acc_full[buf]);
+        }
+        umma_commit(&empty[s]);
+      }
+    }
+  } else {
+    // --------------------------------------------------- epilogue --
+    const int ew = static_cast<int>(warp) - 2;   // 0..7
+    const int g = ew >> 2;                       // accumulator buffer this warpgroup drains
+    const uint32_t quarter = warp & 3u;          // TMEM lanes this warp may access
+    const int key_in_tile = static_cast<int>(quarter * 32 + lane);
+    const uint32_t lane_addr = (quarter * 32u) << 16;
+    const int n_items = n_tiles * C::NG;
+    for (int item = g; item < n_items; item += 2) {
+      const int it = item / C::NG;
+      const int grp = item % C::NG;
+      if (!mbar_wait(&acc_full[g], (item >> 1) & 1, p.budget)) {
+        report_error(p.err, kDevErrTimeout, 130, item);
+        break;
+      }
+      tc_fence_after();
+      const int s = (tile_begin + it) * 128 + key_in_tile;
+      const float ks = s < kv ? __ldg(&p.k_scale[kstart + s]) : 0.f;
+#pragma unroll 1
+      for (int tk = 0; tk < C::GTOK; ++tk) {
+        const int tok = grp * C::GTOK + tk;
+        uint32_t ra[32], rb[32];
+        const uint32_t taddr = tmem + lane_addr + static_cast<uint32_t>(g * C::N + tk * 64);
+        tmem_ld32(taddr, ra);
+        tmem_ld32(taddr + 32, rb);
+        tmem_ld_wait();
+        const float4* w4 = reinterpret_cast<const float4*>(sW + tok * 64);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 wv = w4[j];
+          a0 = fmaf(wv.x, fmaxf(__uint_as_float(ra[4 * j + 0]), 0.f), a0);
+          a1 = fmaf(wv.y, fmaxf(__uint_as_float(ra[4 * j + 1]), 0.f), a1);
+          a2 = fmaf(wv.z, fmaxf(__uint_as_float(ra[4 * j + 2]), 0.f), a2);
+          a3 = fmaf(wv.w, fmaxf(__uint_as_float(ra[4 * j + 3]), 0.f), a3);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 wv = w4[8 + j];
+          a0 = fmaf(wv.x, fmaxf(__uint_as_float(rb[4 * j + 0]), 0.f), a0);
+          a1 = fmaf(wv.y, fmaxf(__uint_as_float(rb[4 * j + 1]), 0.f), a1);
+          a2 = fmaf(wv.z, fmaxf(__uint_as_float(rb[4 * j + 2]), 0.f), a2);
+          a3 = fmaf(wv.w, fmaxf(__uint_as_float(rb[4 * j + 3]), 0.f), a3);
+        }
+        const float acc = (a0 + a1) + (a2 + a3);
+        if (tok < ntok && s <= t_first + tok) {
+          p.scores[static_cast<int64_t>(row0 + tok) * p.ld + s] = acc * ks;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[g]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int TOK>
+cudaError_t launch_tok(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const IndexerParams& p,
+                       cudaStream_t stream) {
+  using C = IdxCfg<TOK>;
+  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  indexer_kernel<TOK><<<grid, kThreads, C::SMEM, stream>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int indexer_tokens_per_cta(int max_q_per_seq) {
+  if (max_q_per_seq >= 8) return 8;
+  if (max_q_per_seq >= 4) return 4;
+  if (max_q_per_seq >= 2) return 2;
+  return 1;
+}
+
+size_t indexer_smem_bytes(int tok) {
+  switch (tok) {
+    case 1: return IdxCfg<1>::SMEM;
+    case 2: return IdxCfg<2>::SMEM;
+    case 4: return IdxCfg<4>::SMEM;
+    default: return IdxCfg<8>::SMEM;
+  }
+}
+
+int indexer_box_rows_q(int tok) {
+  switch (tok) {
+    case 1: return IdxCfg<1>::BOXQ;
+    case 2: return IdxCfg<2>::BOXQ;
+    case 4: return IdxCfg<4>::BOXQ;
+    default: return IdxCfg<8>::BOXQ;
+  }
+}
+
+cudaError_t launch_indexer(int tok, dim3 grid, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                           const IndexerParams& p, cudaStream_t stream) {
+  switch (tok) {
+    case 1: return launch_tok<1>(grid, tmap_q, tmap_k, p, stream);
+    case 2: return launch_tok<2>(grid, tmap_q, tmap_k, p, stream);
+    case 4: return launch_tok<4>(grid, tmap_q, tmap_k, p, stream);
+    case 8: return launch_tok<8>(grid, tmap_q, tmap_k, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dsa

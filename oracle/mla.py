@@ -34,6 +34,20 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def attend(q: np.ndarray, c: np.ndarray, sm_scale: float):
+    """All heads of one token over the gathered entries c [n, 576] (float64)."""
+    H = q.shape[0]
+    if c.shape[0] == 0:
+        return np.zeros((H, VALUE_DIM)), np.full(H, -np.inf)
+    logits = sm_scale * (q @ c.T)                         # [H, n]
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    l = p.sum(axis=1, keepdims=True)
+    o = (p / l) @ c[:, :VALUE_DIM]
+    lse = (m + np.log(l))[:, 0]
+    return o, lse
+
+
 def sparse_token(q: np.ndarray, latent_seq: np.ndarray, idx_row: np.ndarray, sm_scale: float):
     """One query token.
 
@@ -42,17 +56,7 @@ def sparse_token(q: np.ndarray, latent_seq: np.ndarray, idx_row: np.ndarray, sm_
     """
     sel = np.asarray(idx_row, dtype=np.int64)
     sel = sel[sel >= 0]
-    H = q.shape[0]
-    if sel.size == 0:
-        return np.zeros((H, VALUE_DIM)), np.full(H, -np.inf)
-    c = latent_seq[sel]                                   # gather of the selected entries
-    logits = sm_scale * (q @ c.T)                         # [H, n]
-    m = logits.max(axis=1, keepdims=True)
-    p = np.exp(logits - m)
-    l = p.sum(axis=1, keepdims=True)
-    o = (p / l) @ c[:, :VALUE_DIM]
-    lse = (m + np.log(l))[:, 0]
-    return o, lse
+    return attend(q, latent_seq[sel], sm_scale)          # gather of the selected entries
 
 
 def dense_masked(q: np.ndarray, latent_seq: np.ndarray, idx_row: np.ndarray, t: int,
@@ -78,26 +82,34 @@ def dense_masked(q: np.ndarray, latent_seq: np.ndarray, idx_row: np.ndarray, t: 
 def sparse(inputs, idx: np.ndarray, rows=None):
     """Sparse MLA for query rows ``rows`` of a ``DSAInputs`` batch.
 
-    ``idx`` is the [n_q, k] index array (sequence-relative positions, -1 pad).
-    Returns {row: (o [H, 512] float64, lse [H] float64)}.
+    ``idx`` is an [n_rows, k] index array (sequence-relative positions, -1 or
+    out-of-range = skipped), row i of ``idx`` belonging to query row rows[i]
+    (default: all rows, idx[r] for row r).  Returns {row: (o [H, 512], lse [H])}.
     """
     b = inputs.batch
-    rows = range(b.total_q) if rows is None else rows
+    rows = list(range(b.total_q)) if rows is None else [int(r) for r in rows]
     out = {}
-    for r in rows:
-        r = int(r)
+    for i, r in enumerate(rows):
         seq = int(b.q_seq[r])
         k0 = int(b.kv_start[seq])
         kv = int(b.kv_len[seq])
-        sel = np.asarray(idx[r], dtype=np.int64)
-        used = np.unique(sel[sel >= 0])
-        lat = np.zeros((kv, inputs.latent.shape[1]))
-        lat[used] = bf16_to_f64(inputs.latent[k0 + used])
+        sel = np.asarray(idx[i], dtype=np.int64)
+        sel = sel[(sel >= 0) & (sel < kv)]
+        c = bf16_to_f64(inputs.latent[k0 + sel])
         q = bf16_to_f64(inputs.q_mla[r])
-        out[r] = sparse_token(q, lat, sel, inputs.sm_scale)
+        out[r] = attend(q, c, inputs.sm_scale)
     return out
 
 
 def flops_per_token(n_heads: int, n_sel: int, latent_dim: int = 576, value_dim: int = VALUE_DIM) -> int:
     """Tensor-core work of one token: QK^T over 576 dims and PV over 512."""
     return 2 * n_heads * n_sel * (latent_dim + value_dim)
+
+
+def bf16_output(o: np.ndarray) -> np.ndarray:
+    """The output in the path's storage format: fp64 -> fp32 -> bf16, round to
+    nearest even (the attention output is bf16).  Returned as float64 values."""
+    f = np.ascontiguousarray(o, dtype=np.float32)
+    u = f.view(np.uint32)
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)) << np.uint32(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)

@@ -1,0 +1,100 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry point,
+sizes workspaces, describes statuses and rejects bad arguments before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import long_context_sparse_lightning_b200 as dsa
+from long_context_sparse_lightning_b200 import _BatchC
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dsa.library()
+    names = declared_functions()
+    assert set(names) == set(dsa.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert dsa.version() == 100
+    lib = dsa.library()
+    for code in range(7):
+        assert lib.dsa_status_string(code).decode()
+    assert lib.dsa_status_string(99) == b"unknown status"
+
+
+def _host_batch(B=2, total_q=10, max_q=6, max_kv=100, total_keys=180):
+    c = _BatchC()
+    c.num_seqs, c.total_q, c.max_q_per_seq, c.max_kv_len, c.total_keys = B, total_q, max_q, max_kv, total_keys
+    c.cu_q = c.kv_len = c.kv_start = 0x1000   # never dereferenced on the host
+    return c
+
+
+def test_workspace_sizes():
+    lib = dsa.library()
+    c = _host_batch()
+    ref = ctypes.byref(c)
+    assert lib.dsa_workspace_size(dsa.OP_INDEXER, ref, 64, 16) == 256
+    assert lib.dsa_workspace_size(dsa.OP_TOPK, ref, 64, 16) == 256
+    fwd = lib.dsa_workspace_size(dsa.OP_FORWARD, ref, 64, 16)
+    assert fwd >= 256 + 10 * 100 * 4
+    assert lib.dsa_workspace_size(dsa.OP_FORWARD, ref, 4096, 16) == 0       # k_sel too large
+    assert lib.dsa_workspace_size(dsa.OP_SPARSE_MLA, ref, 64, 256) == 0     # too many heads
+    bad = _host_batch(B=0)
+    assert lib.dsa_workspace_size(dsa.OP_TOPK, ctypes.byref(bad), 64, 16) == 0
+
+
+def test_rejections_happen_before_any_launch():
+    lib = dsa.library()
+    c = _host_batch()
+    ref = ctypes.byref(c)
+    P = ctypes.c_void_p
+    fake = P(0x10000)                   # aligned, never dereferenced
+    # null pointers
+    assert lib.dsa_indexer_scores(ref, None, fake, fake, fake, fake, fake, 100, fake, 4096, None) == 1
+    assert lib.dsa_topk(ref, fake, 100, 64, None, fake, 4096, None) == 1
+    # misaligned pointer
+    assert lib.dsa_topk(ref, P(0x10004), 100, 64, fake, fake, 4096, None) == 1
+    # leading dimension too small / not a multiple of 4
+    assert lib.dsa_topk(ref, fake, 99, 64, fake, fake, 4096, None) == 1
+    assert lib.dsa_topk(ref, fake, 102, 64, fake, fake, 4096, None) == 1
+    # unsupported k_sel / heads
+    assert lib.dsa_topk(ref, fake, 100, 4096, fake, fake, 4096, None) == 2
+    assert lib.dsa_sparse_mla(ref, fake, 200, fake, fake, 64, 0.07, fake, None, fake, 4096, None) == 2
+    # bad scale
+    assert lib.dsa_sparse_mla(ref, fake, 16, fake, fake, 64, -1.0, fake, None, fake, 4096, None) == 1
+    # workspace too small
+    assert lib.dsa_topk(ref, fake, 100, 64, fake, fake, 16, None) == 4
+    need = lib.dsa_workspace_size(dsa.OP_FORWARD, ref, 64, 16)
+    assert lib.dsa_forward(ref, fake, fake, fake, fake, fake, 64, fake, 16, fake, 0.07, fake, fake, None, fake,
+                           need - 1, None) == 4
+    # inconsistent batch
+    bad = _host_batch(max_q=20)          # max_q_per_seq > total_q
+    assert lib.dsa_topk(ctypes.byref(bad), fake, 100, 64, fake, fake, 4096, None) == 1
+
+
+def test_empty_batch_is_a_no_op():
+    lib = dsa.library()
+    c = _host_batch(total_q=0, max_q=0)
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.dsa_topk(ctypes.byref(c), fake, 100, 64, fake, fake, 4096, None) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(dsa, "LIB_PATH", "/nonexistent/libdsa.so")
+    monkeypatch.setattr(dsa, "_LIB", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        dsa.library()
