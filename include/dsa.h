@@ -144,6 +144,39 @@ DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, co
                          const void* kv, float sm_scale, int32_t* idx, void* out, float* lse, void* ws,
                          size_t ws_bytes, dsa_stream_t stream);
 
+/* Sparse MLA without a caller workspace -- for callers that cannot allocate
+ * device memory.  (The pages have no counterpart to this entry point; it is a
+ * deployment convenience.)
+ *
+ * Who needs it: code that does not own an allocator, e.g. a plugin inside a
+ * host engine that may only use the buffers the engine hands it, or a
+ * latency-critical loop where cudaMalloc's implicit device synchronisation is
+ * not acceptable.  Such callers still provide q, kv, idx, out and lse exactly
+ * as for dsa_sparse_mla; the split-selection partial results that
+ * dsa_sparse_mla keeps in `ws` live instead in a library-owned device array of
+ * DSA_NO_ALLOC_SCRATCH_BYTES (32 MiB), which every GPU that loads the library
+ * holds until the process exits.  The call itself performs no cudaMalloc,
+ * cudaFree or other allocation.
+ *
+ *   - Batches whose partial results need more than the scratch array (more
+ *     than 256 B + total_q * nsplit * 128 * 2052 B, rounded) return
+ *     DSA_ERR_WORKSPACE before anything is launched; use dsa_sparse_mla then.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps the previous
+ *     call's contents; each call clears the error word it needs at the start.
+ *     Calls whose work overlaps on the GPU (different streams, no ordering)
+ *     race on the array and must be serialised by the caller.
+ *   - Device-side error statuses (bounded-wait timeouts) are recorded in the
+ *     array and are not reported to the caller; use dsa_sparse_mla with a
+ *     workspace and dsa_check_device_error when they are needed.
+ * Arguments and results are otherwise those of dsa_sparse_mla. */
+#define DSA_NO_ALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+DSA_API dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* batch, const void* q, int32_t n_heads,
+                                             const void* kv, const int32_t* idx, int32_t k_sel, float sm_scale,
+                                             void* out, float* lse, dsa_stream_t stream);
+
 /* Synchronise `stream`, read the device error word of `ws`, clear it, and
  * return DSA_OK, DSA_ERR_DEVICE_TIMEOUT or DSA_ERR_DEVICE_BOUNDS (or
  * DSA_ERR_CUDA if the stream reports an error).  `site` / `info`, if not NULL,

@@ -42,6 +42,7 @@ EXPORTS = [
     "dsa_topk",
     "dsa_sparse_mla",
     "dsa_forward",
+    "dsa_sparse_mla_no_alloc",
     "dsa_check_device_error",
     "dsa_status_string",
     "dsa_version",
@@ -90,6 +91,8 @@ def _lib():
         lib.dsa_sparse_mla.restype = ctypes.c_int
         lib.dsa_forward.argtypes = [BP, P, P, P, P, P, I32, P, I32, P, F, P, P, P, P, SZ, P]
         lib.dsa_forward.restype = ctypes.c_int
+        lib.dsa_sparse_mla_no_alloc.argtypes = [BP, P, I32, P, P, I32, F, P, P, P]
+        lib.dsa_sparse_mla_no_alloc.restype = ctypes.c_int
         lib.dsa_check_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
         lib.dsa_check_device_error.restype = ctypes.c_int
         lib.dsa_status_string.argtypes = [ctypes.c_int]
