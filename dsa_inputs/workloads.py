@@ -93,6 +93,17 @@ WORKLOADS: dict[str, Workload] = {
             description="8 sequences x 2 query tokens at 131072 context, top-2048, 128 MLA heads",
             num_seqs=8, q_len=2, kv_len=131072, k_sel=2048, n_heads=128,
         ),
+        # smaller shapes of the same kinds, for profiling captures
+        Workload(
+            name="chunked_prefill_32k_512",
+            description="1 sequence, 512 new queries ending at position 32767 (32768 keys), top-2048, 128 MLA heads",
+            num_seqs=1, q_len=512, kv_len=32768, k_sel=2048, n_heads=128, heavy_frac=0.05,
+        ),
+        Workload(
+            name="decode_16x32k",
+            description="16 sequences x 1 query token at 32768 context, top-2048, 128 MLA heads",
+            num_seqs=16, q_len=1, kv_len=32768, k_sel=2048, n_heads=128,
+        ),
     ]
 }
 

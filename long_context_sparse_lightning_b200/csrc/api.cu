@@ -106,6 +106,17 @@ size_t mla_part_bytes(const dsa_batch_t* b, int k_sel) {
   return align_up(rows * 512 * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
 }
 
+bool mla_copy(const dsa_batch_t* b, int k_sel) {
+  return dsa::mla_use_fp16_copy(b->total_q, b->max_kv_len, b->total_keys, k_sel);
+}
+
+// partial results + (prefill-shaped batches) the fp16 copy of the latent cache
+size_t mla_ws_bytes(const dsa_batch_t* b, int k_sel) {
+  size_t n = mla_part_bytes(b, k_sel);
+  if (mla_copy(b, k_sel)) n += align_up(static_cast<size_t>(b->total_keys) * 576 * 2, 256);
+  return n;
+}
+
 // ----------------------------------------------------------------- stages --
 dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q_scale, const float* w,
                          const void* k_fp8, const float* k_scale, float* scores, int64_t ld, uint32_t* err,
@@ -187,7 +198,21 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   const int64_t gx = int64_t(2) * b->max_q_per_seq * sp.nsplit;
   if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
-  if (dsa::launch_sparse_mla(grid, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (mla_copy(b, k_sel)) {
+    uint16_t* kv16 = reinterpret_cast<uint16_t*>(part + mla_part_bytes(b, k_sel));
+    const int64_t n = b->total_keys * 576;
+    if (dsa::launch_latent_to_fp16(static_cast<const uint16_t*>(kv), kv16, n, stream) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    CUtensorMap ml, mr;
+    if (!make_tmap_2d(&ml, kv16, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(b->total_keys), 576, 1, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&mr, kv16, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(b->total_keys), 576, 1, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
+      return DSA_ERR_CUDA;
+    if (dsa::launch_sparse_mla_tma(grid, p, ml, mr, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  } else if (dsa::launch_sparse_mla(grid, p, stream) != cudaSuccess) {
+    return DSA_ERR_CUDA;
+  }
   if (sp.nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }
@@ -222,11 +247,11 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, 
       return kHeaderBytes;
     case DSA_OP_SPARSE_MLA:
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
-      return kHeaderBytes + mla_part_bytes(batch, k_sel);
+      return kHeaderBytes + mla_ws_bytes(batch, k_sel);
     case DSA_OP_FORWARD: {
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
       const size_t scores = align_up(static_cast<size_t>(batch->total_q) * forward_ld(batch) * sizeof(float), 256);
-      return kHeaderBytes + scores + mla_part_bytes(batch, k_sel);
+      return kHeaderBytes + scores + mla_ws_bytes(batch, k_sel);
     }
   }
   return 0;
@@ -267,7 +292,7 @@ dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_h
   if (s != DSA_OK) return s;
   if ((s = check_mla_args(q, n_heads, kv, k_sel, sm_scale, out)) != DSA_OK) return s;
   if (idx == nullptr) return DSA_ERR_INVALID_ARG;
-  if ((s = check_ws(ws, ws_bytes, kHeaderBytes + mla_part_bytes(batch, k_sel))) != DSA_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes + mla_ws_bytes(batch, k_sel))) != DSA_OK) return s;
   if (batch->total_q == 0) return DSA_OK;
   return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, static_cast<uint8_t*>(ws) + kHeaderBytes,
                  static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));

@@ -47,30 +47,41 @@ cudaError_t launch_topk(int max_kv_len, dim3 grid, const TopkParams& p, cudaStre
 
 // ------------------------------------------------------------- sparse MLA --
 struct MlaParams {
-  const int32_t* cu_q;
-  const int32_t* kv_len;
-  const int64_t* kv_start;
-  const uint16_t* q;        // bf16 [total_q, H, 576]
-  const uint16_t* kv;       // bf16 [total_keys, 576]
-  const int32_t* idx;       // [total_q, k_sel]
-  int64_t total_keys;
-  int32_t k_sel;
-  int32_t n_heads;
-  float scale_log2;         // sm_scale * log2(e)
-  uint16_t* out;            // bf16 [total_q, H, 512]
-  float* lse;               // [total_q, H] or nullptr
-  float* part_o;            // [total_q, nsplit, 128, 512] fp32 when nsplit > 1
-  float* part_lse;          // [total_q, nsplit, 128]
-  int32_t nsplit;
-  int32_t keys_per_split;   // multiple of 64
-  uint32_t* err;
-  long long budget;
+  const int32_t* cu_q = nullptr;
+  const int32_t* kv_len = nullptr;
+  const int64_t* kv_start = nullptr;
+  const uint16_t* q = nullptr;        // bf16 [total_q, H, 576]
+  const uint16_t* kv = nullptr;       // bf16 [total_keys, 576]
+  const int32_t* idx = nullptr;       // [total_q, k_sel]
+  int64_t total_keys = 0;
+  int32_t k_sel = 0;
+  int32_t n_heads = 0;
+  float scale_log2 = 0.f;             // sm_scale * log2(e)
+  uint16_t* out = nullptr;            // bf16 [total_q, H, 512]
+  float* lse = nullptr;               // [total_q, H] or nullptr
+  float* part_o = nullptr;            // [total_q, nsplit, 128, 512] fp32 when nsplit > 1
+  float* part_lse = nullptr;          // [total_q, nsplit, 128]
+  int32_t nsplit = 1;
+  int32_t keys_per_split = 0;         // multiple of 64
+  uint32_t* err = nullptr;
+  long long budget = 2000000000LL;
 };
 
 int mla_num_splits(int total_q, int max_q_per_seq, int num_seqs, int k_sel);
 int mla_keys_per_split(int k_sel, int nsplit);
+// Gather from an fp16 copy of the latent cache (made once per call) when the
+// selections reuse each latent row often enough to amortise the copy.
+bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_sel);
 size_t mla_smem_bytes();
+// Selected rows gathered with 16-byte loads and converted to fp16 on the way
+// into shared memory (no extra buffers).
 cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, cudaStream_t stream);
+// Selected rows gathered by TMA from `kv16`, an fp16 copy of the latent cache
+// described by the two tensor maps (64-column / 128-byte-swizzled boxes for the
+// latent dims, 32-column / 64-byte-swizzled boxes for the RoPE dims).
+cudaError_t launch_sparse_mla_tma(dim3 grid, const MlaParams& p, const CUtensorMap& map_lat,
+                                  const CUtensorMap& map_rope, cudaStream_t stream);
+cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream);
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream);
 
 }  // namespace dsa

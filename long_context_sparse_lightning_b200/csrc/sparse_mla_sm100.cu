@@ -1,5 +1,5 @@
-// Sparse MLA in MQA mode on sm_100a (tcgen05, TMEM accumulators, a CTA pair
-// per query token).
+// Sparse MLA in MQA mode on sm_100a (tcgen05, TMEM operands and accumulators,
+// a CTA pair per query token).
 //
 // "DeepSeek V3.2 稀疏注意力" (embedding DSA in MLA) and "NSA 与 DSA" §3.1: all
 // query heads of a token share the same selected latent entries c_s (576-d =
@@ -7,32 +7,43 @@
 // tile of entries feeds every head:
 //     o[h] = sum_i softmax_i(sm_scale * q[h] . c[s_i]) * c[s_i][0:512].
 //
-// Layout of the work: a cluster of two CTAs handles one token (or one split of
-// its selected entries).  CTA r owns latent dims [256r, 256r+256) and RoPE
-// dims [512+32r, 512+32r+32) -- 288 of the 576 score dims and 256 of the 512
-// value dims -- so the 128 x 512 fp32 output accumulator is split 256 TMEM
-// columns per CTA and every latent byte is gathered exactly once per pair.
+// Work split: a cluster of two CTAs handles one token (or one split of its
+// selection).  CTA r owns score dims [256r, 256r+256) U [512+32r, 544+32r)
+// (288 of 576) and value dims [256r, 256r+256), so the 128 x 512 fp32 output
+// accumulator is split 256 TMEM columns per CTA and each selected latent row is
+// fetched once per pair.
+//
+// Tensor memory of one CTA (512 columns x 128 lanes, lane = head):
+//   O [0,256) fp32, S [256,320) fp32, P [320,352) fp16 pairs, Q [352,496) fp16 pairs.
+// Q and P are the A operands of their MMAs straight from TMEM, so the only
+// shared-memory operand traffic is the gathered tile (B operand of both MMAs:
+// K-major for Q.C^T, MN-major for P.V).
+//
 // Per tile of 64 selected entries:
-//   producers (6 warps)  gather this CTA's 288 dims of each selected row with
-//                        16-byte loads, convert bf16 -> fp16 (exact for the
-//                        normal fp16 range) and store them 128/64-byte
-//                        swizzled; the same tile serves QK^T as a K-major B
-//                        operand and PV as an MN-major B operand;
-//   MMA warp             S_r = Q_r . C_r^T (M=128 heads, N=64, K=288, fp16 in,
-//                        fp32 in TMEM), later O_r += P . V_r (N=256);
-//   softmax (4 warps)    thread h owns head h: exchanges its 64 partial scores
-//                        with the partner CTA through distributed shared memory,
-//                        adds them (both CTAs get bit-identical S), runs the
-//                        online softmax in the log2 domain with a lazily
-//                        refreshed running max (rescale of O only when the max
-//                        grows by more than 2^8), writes P as fp16.
-// P is fp16 rather than bf16: with bf16 probabilities the rounding noise alone
-// costs ~1e-3 mean relative error on the bf16 output; fp16 keeps it ~1e-4.
+//   gather     fp16 copy of the latent cache + TMA gather4 (prefill: rows are
+//              reused across many tokens), or 6 producer warps copying bf16 rows
+//              with 16-byte cp.async into place and converting them to fp16 in
+//              shared memory (decode); 4-stage ring;
+//   MMA warp   S_r = Q_r . C_r^T (M=128, N=64, K=288) then O_r += P . V_r (N=256);
+//   softmax    8 warps, two per TMEM lane quarter, each half owning 32 of the 64
+//              columns: each warp ships its 2 KB of partial scores (fp16; both
+//              CTAs then add the same two rounded numbers, so S is bit-identical
+//              in both) to the peer with one bulk shared-to-shared copy, one tile
+//              ahead of its own use so the transfer overlaps a whole iteration;
+//              row max across the halves through shared memory; online softmax
+//              in log2 units with a lazily refreshed max (O rescaled in TMEM only
+//              when the max grows by more than 2^8); P stored to TMEM as fp16.
+//   MMA order  Q.C^T runs two tiles ahead of P.V.
+// fp16 rather than bf16 inside the MMAs: with bf16 probabilities the rounding
+// noise costs ~1e-3 mean relative error on the bf16 output; fp16 keeps ~1e-4.
+// The conversion of q and the latent entries is exact in the normal fp16 range.
 //
 // Decode shapes split a token's selection over several pairs; each writes a
 // normalised partial output and its log-sum-exp, merged by mla_combine_kernel.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <cstring>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -40,46 +51,51 @@
 namespace dsa {
 namespace {
 
-constexpr int kProdWarps = 6;
-constexpr int kProdThreads = kProdWarps * 32;
-constexpr int kMmaWarp = kProdWarps;              // warp 8
-constexpr int kThreads = (kProdWarps + 1 + 4) * 32;
 constexpr int kTileKeys = 64;
-constexpr int kUnitsPerRow = 36;                  // 16-byte units per gathered row half (288 dims)
-constexpr int kTileUnits = kTileKeys * kUnitsPerRow;
-constexpr int kUnitsPerThread = kTileUnits / kProdThreads;   // 9
-static_assert(kTileUnits % kProdThreads == 0, "");
-constexpr int kQUnits = 128 * kUnitsPerRow;
-constexpr int kQUnitsPerThread = kQUnits / kProdThreads;     // 18
-
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr int OFF_Q = 0;                 // 4 x [128 x 128 B] SW128 + [128 x 64 B] SW64
-constexpr int Q_ROPE = 65536;
-constexpr int OFF_KV = 73728;            // 2 stages x 36864
-constexpr int KV_STAGE = 36864;
+constexpr int kStages = 4;
+constexpr int KV_STAGE = 36864;          // 64 rows x (4 x 128 B latent + 64 B RoPE)
 constexpr int KV_ROPE = 32768;
-constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;     // 147456: 2 x [128 x 128 B] SW128 fp16
-constexpr int P_BYTES = 16384;
-constexpr int OFF_X = OFF_P + 2 * P_BYTES;       // 180224: incoming partial S, 128 rows x 272 B
-constexpr int X_PITCH = 272;
-constexpr int OFF_IDX = OFF_X + 128 * X_PITCH;   // 215040
-constexpr int OFF_BAR = OFF_IDX + 2048 * 4;      // 223232
-constexpr int OFF_MISC = OFF_BAR + 128;
+constexpr int XBLK = 2048;               // one softmax warp's partial scores: 32 heads x 32 keys fp16
+constexpr int XBUF = 8 * XBLK;           // one tile's partial scores of all 8 softmax warps
+
+constexpr uint32_t TM_O = 0;
+constexpr uint32_t TM_S = 256;
+constexpr uint32_t TM_P = 320;
+constexpr uint32_t TM_Q = 352;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr int OFF_KV = 0;
+constexpr int OFF_STG = kStages * KV_STAGE;          // 147456: outgoing partial scores, 2 buffers
+constexpr int OFF_X = OFF_STG + 2 * XBUF;            // 180224: incoming partial scores, 2 buffers
+constexpr int OFF_IDX = OFF_X + 2 * XBUF;            // 212992: int32[2048]
+constexpr int OFF_VALID = OFF_IDX + 2048 * 4;        // 221184: uint32[64] validity bits
+constexpr int OFF_RED = OFF_VALID + 64 * 4;          // 221440: float[2][2][128] row maxima, float[2][128] sums
+constexpr int OFF_BAR = OFF_RED + 6 * 128 * 4;       // 224512
+constexpr int OFF_MISC = OFF_BAR + 256;
 constexpr int kSmem = OFF_MISC + 64 + 1024;
-constexpr uint32_t kTmemCols = 512;              // O: cols [0,256), S: [256,384)
+
+constexpr int kUnitsPerRow = 36;                     // 16-byte units of a row's 288-dim half
+constexpr int kTileUnits = kTileKeys * kUnitsPerRow; // 2304
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[2];
-  uint64_t kv_empty[2];
-  uint64_t s_full[2];
-  uint64_t s_empty[2];
-  uint64_t x_full;
-  uint64_t x_free;
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full, s_empty;
+  uint64_t x_full[2], x_free[2];
+  uint64_t p_full, pv_done;
+  uint64_t red;            // the two column halves' row maxima / sums are in shared memory
 };
-static_assert(sizeof(Bars) <= 128, "");
+static_assert(sizeof(Bars) <= 256, "");
+
+template <bool TMA>
+struct Cfg {
+  static constexpr int NPROD = TMA ? 1 : 6;          // producer warps
+  static constexpr int MMA_WARP = NPROD;
+  static constexpr int SOFT0 = NPROD + 1;            // 8 softmax warps follow
+  static constexpr int THREADS = (NPROD + 1 + 8) * 32;
+  static constexpr int UNITS = TMA ? 1 : kTileUnits / (NPROD * 32);   // 12 per producer thread
+};
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   const float lo = __uint_as_float(w << 16);
@@ -99,19 +115,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// smem offset (within a 288-dim row group) of 16-byte unit u of row j:
-// units 0..31 = latent dims (4 chunks of 8 units, 128-byte swizzle),
-// units 32..35 = RoPE dims (64-byte swizzle).
-__device__ __forceinline__ uint32_t tile_unit_offset(int j, int u, int chunk_bytes, int rope_off) {
-  if (u < 32) {
-    const int c = u >> 3, cu = u & 7;
-    return c * chunk_bytes + j * 128 + ((cu ^ (j & 7)) << 4);
-  }
-  const int ru = u - 32;
-  return rope_off + j * 64 + ((ru ^ ((j >> 1) & 3)) << 4);
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaParams p) {
+// Global dim of 16-byte unit u (0..35) of CTA r's 288-dim half of a 576-d row.
+__device__ __forceinline__ int unit_dim(int u, uint32_t r) {
+  return u < 32 ? static_cast<int>(r) * 256 + u * 8 : 512 + static_cast<int>(r) * 32 + (u - 32) * 8;
+}
+
+// Shared-memory offset of unit u of row j inside a stage: units 0..31 form four
+// 64-dim chunks (8 KB each, 128-byte swizzle), units 32..35 the RoPE chunk
+// (64-byte swizzle) -- the layouts TMA writes for 128/64-byte boxes.
+__device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
+  if (u < 32) {
+    const int c = u >> 3, cu = u & 7;
+    return c * 8192 + j * 128 + ((cu ^ (j & 7)) << 4);
+  }
+  const int ru = u - 32;
+  return KV_ROPE + j * 64 + ((ru ^ ((j >> 1) & 3)) << 4);
+}
+
+template <bool TMA>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1)
+    sparse_mla_kernel(const MlaParams p, const __grid_constant__ CUtensorMap map_lat,
+                      const __grid_constant__ CUtensorMap map_rope) {
+  using C = Cfg<TMA>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -122,16 +152,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
   const int b = blockIdx.y;
   const int q0 = __ldg(&p.cu_q[b]);
   const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
-  // Every early exit below depends only on launch indices and device inputs
-  // that do not change during the kernel, so both CTAs of a pair take it
-  // together; a one-sided exit would leave the partner in barrier.cluster.
+  // Every early exit depends only on launch indices and on device inputs that
+  // do not change during the kernel, so both CTAs of a pair take it together
+  // (a one-sided exit would leave the peer waiting in barrier.cluster).
   if (tok >= q_len) return;
   const int row = q0 + tok;
   const int kv = __ldg(&p.kv_len[b]);
   const int64_t kstart = __ldg(&p.kv_start[b]);
   if (q_len > kv || kstart < 0 || kstart + kv > p.total_keys) {
     if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 301, b);
-    return;                             // both CTAs of the pair take this branch
+    return;
   }
   const int H = p.n_heads;
   const int e_begin = split * p.keys_per_split;
@@ -139,11 +169,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
 
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = sm + OFF_Q;
   uint8_t* sKV = sm + OFF_KV;
-  uint8_t* sP = sm + OFF_P;
-  float* sX = reinterpret_cast<float*>(sm + OFF_X);
   int32_t* sIdx = reinterpret_cast<int32_t*>(sm + OFF_IDX);
+  uint32_t* sValid = reinterpret_cast<uint32_t*>(sm + OFF_VALID);
+  float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
   Bars* bar = reinterpret_cast<Bars*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   int32_t* s_last = reinterpret_cast<int32_t*>(sm + OFF_MISC + 4);
@@ -152,39 +181,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
   const uint32_t lane = lane_id();
   const int tid = threadIdx.x;
 
-  // ---- selected positions of this split; invalid ones become -1 ----
+  // ---- this split's selected positions (invalid -> -1) and per-32 validity bits ----
   if (tid == 0) *s_last = -1;
   __syncthreads();
   const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
   int my_last = -1;
-  for (int j = tid; j < 2048; j += kThreads) {
+  for (int j = tid; j < 2048; j += C::THREADS) {
     int v = -1;
     if (j < e_count) {
       v = __ldg(&idx_row[j]);
       if (v < 0 || v >= kv) v = -1;
     }
     sIdx[j] = v;
+    const uint32_t bits = __ballot_sync(0xffffffffu, v >= 0);
+    if (lane == 0) sValid[j >> 5] = bits;
     if (v >= 0) my_last = j;
   }
   if (my_last >= 0) atomicMax(s_last, my_last);
 
   if (tid == 0) {
-    mbar_init(&bar->q_full, kProdWarps);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->kv_full[i], kProdWarps);
-      mbar_init(&bar->kv_empty[i], 1);
-      mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->s_empty[i], 4);
+    mbar_init(&bar->q_full, 8);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar->kv_full[s], TMA ? 1 : C::NPROD);
+      mbar_init(&bar->kv_empty[s], 1);
     }
-    mbar_init(&bar->x_full, 128);
-    mbar_init(&bar->x_free, 128);
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->s_empty, 8);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->p_full[i], 128);
-      mbar_init(&bar->pv_done[i], 1);
+      mbar_init(&bar->x_full[i], 8);    // one expect_tx arrival per receiving warp + 16 KB of bulk copies
+      mbar_init(&bar->x_free[i], 8);    // one remote arrival per peer warp once it has read the buffer
     }
+    mbar_init(&bar->p_full, 8);
+    mbar_init(&bar->pv_done, 1);
+    mbar_init(&bar->red, 256);
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -195,264 +227,371 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
   const int n_ent = *s_last + 1;
   const int n_tiles = (n_ent + kTileKeys - 1) / kTileKeys;
 
-  if (warp < kProdWarps) {
-    // ------------------------------------------ gather + convert producers --
-    if (n_tiles > 0) {
-      // Q_r: this token's 128 head rows (rows >= H are zero)
-      {
-        const uint16_t* qrow = p.q + static_cast<int64_t>(row) * H * 576;
-#pragma unroll 4
-        for (int m = 0; m < kQUnitsPerThread; ++m) {
-          const int g = tid + m * kProdThreads;
-          const int h = g / kUnitsPerRow, u = g % kUnitsPerRow;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (h < H) {
-            const int dim = u < 32 ? static_cast<int>(rank) * 256 + u * 8 : 512 + static_cast<int>(rank) * 32 + (u - 32) * 8;
-            v = cvt_unit(__ldg(reinterpret_cast<const uint4*>(qrow + h * 576 + dim)));
+  if (warp < C::NPROD) {
+    // ------------------------------------------------------------ producers --
+    if constexpr (TMA) {
+      if (n_tiles > 0 && elect_one()) {
+        prefetch_tmap(&map_lat);
+        prefetch_tmap(&map_rope);
+        for (int i = 0; i < n_tiles; ++i) {
+          const int st = i % kStages;
+          if (!mbar_wait(&bar->kv_empty[st], ((i / kStages) & 1) ^ 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 310, i);
+            break;
           }
-          *reinterpret_cast<uint4*>(sQ + tile_unit_offset(h, u, 16384, Q_ROPE)) = v;
+          mbar_arrive_expect_tx(&bar->kv_full[st], KV_STAGE);
+          uint8_t* base = sKV + st * KV_STAGE;
+          const int* e = sIdx + i * kTileKeys;
+#pragma unroll 1
+          for (int g4 = 0; g4 < 16; ++g4) {
+            const int y0 = static_cast<int>(kstart + max(e[4 * g4 + 0], 0));
+            const int y1 = static_cast<int>(kstart + max(e[4 * g4 + 1], 0));
+            const int y2 = static_cast<int>(kstart + max(e[4 * g4 + 2], 0));
+            const int y3 = static_cast<int>(kstart + max(e[4 * g4 + 3], 0));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              tma_gather4(base + c * 8192 + g4 * 512, &map_lat, &bar->kv_full[st],
+                          static_cast<int>(rank) * 256 + c * 64, y0, y1, y2, y3);
+            }
+            tma_gather4(base + KV_ROPE + g4 * 256, &map_rope, &bar->kv_full[st], 512 + static_cast<int>(rank) * 32,
+                        y0, y1, y2, y3);
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->q_full);
       }
-      const uint16_t* kvbase = p.kv + kstart * 576;
-      uint4 bufA[kUnitsPerThread], bufB[kUnitsPerThread];
-      auto issue = [&](int tile, uint4 (&buf)[kUnitsPerThread]) {
+    } else {
+      if (n_tiles > 0) {
+        // cp.async each 16-byte unit straight to its swizzled slot (bf16), then
+        // convert the thread's own units to fp16 in place; two tiles ahead.
+        const uint16_t* kvbase = p.kv + kstart * 576;
+        bool ok = true;
+        auto issue = [&](int tile) {
+          const int st = tile % kStages;
+          if (ok && !mbar_wait(&bar->kv_empty[st], ((tile / kStages) & 1) ^ 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 311, tile);
+            ok = false;
+          }
+          if (ok) {
+            const uint32_t base = smem_u32(sKV + st * KV_STAGE);
 #pragma unroll
-        for (int m = 0; m < kUnitsPerThread; ++m) {
-          const int g = tid + m * kProdThreads;
-          const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
-          const int s = sIdx[tile * kTileKeys + j];
-          const int pos = s >= 0 ? s : 0;
-          const int dim = u < 32 ? static_cast<int>(rank) * 256 + u * 8 : 512 + static_cast<int>(rank) * 32 + (u - 32) * 8;
-          buf[m] = __ldg(reinterpret_cast<const uint4*>(kvbase + static_cast<int64_t>(pos) * 576 + dim));
-        }
-      };
-      bool ok = true;
-      auto commit = [&](int tile, const uint4 (&buf)[kUnitsPerThread]) {
-        const int st = tile & 1;
-        if (ok && !mbar_wait(&bar->kv_empty[st], ((tile >> 1) & 1) ^ 1, p.budget)) {
-          report_error(p.err, kDevErrTimeout, 310, tile);
-          ok = false;
-        }
-        if (!ok) return;
-        uint8_t* base = sKV + st * KV_STAGE;
+            for (int m = 0; m < C::UNITS; ++m) {
+              const int g = tid + m * C::NPROD * 32;
+              const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
+              const int s = sIdx[tile * kTileKeys + j];
+              const int pos = s >= 0 ? s : 0;
+              cp_async_16(base + tile_unit_offset(j, u), kvbase + static_cast<int64_t>(pos) * 576 + unit_dim(u, rank));
+            }
+          }
+          cp_async_commit();
+        };
+        auto convert = [&](int tile) {
+          uint8_t* base = sKV + (tile % kStages) * KV_STAGE;
 #pragma unroll
-        for (int m = 0; m < kUnitsPerThread; ++m) {
-          const int g = tid + m * kProdThreads;
-          const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
-          *reinterpret_cast<uint4*>(base + tile_unit_offset(j, u, 8192, KV_ROPE)) = cvt_unit(buf[m]);
+          for (int m = 0; m < C::UNITS; ++m) {
+            const int g = tid + m * C::NPROD * 32;
+            uint4* q = reinterpret_cast<uint4*>(base + tile_unit_offset(g / kUnitsPerRow, g % kUnitsPerRow));
+            *q = cvt_unit(*q);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->kv_full[tile % kStages]);
+        };
+        // convert tile i before waiting for tile i+2's ring slot: that slot is
+        // freed by P.V of tile i-2, which runs after Q.C^T of tile i, which
+        // needs tile i converted
+        issue(0);
+        if (n_tiles > 1) issue(1);
+        for (int i = 0; i < n_tiles; ++i) {
+          if (i + 1 < n_tiles) {
+            cp_async_wait<1>();
+          } else {
+            cp_async_wait<0>();
+          }
+          if (!ok) break;
+          convert(i);
+          if (i + 2 < n_tiles) issue(i + 2);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->kv_full[st]);
-      };
-      issue(0, bufA);
-      for (int i = 0; i < n_tiles && ok; i += 2) {
-        if (i + 1 < n_tiles) issue(i + 1, bufB);
-        commit(i, bufA);
-        if (i + 1 < n_tiles) {
-          if (i + 2 < n_tiles) issue(i + 2, bufA);
-          commit(i + 1, bufB);
-        }
+        cp_async_wait<0>();
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------- MMA issuer --
+  } else if (warp == C::MMA_WARP) {
+    // ----------------------------------------------------------- MMA issuer --
     if (n_tiles > 0 && elect_one()) {
-      constexpr uint32_t idesc_qk = idesc_f32acc(0, 0, 128, 64, 0, 0);     // fp16 x fp16, K-major both
+      constexpr uint32_t idesc_qk = idesc_f32acc(0, 0, 128, 64, 0, 0);     // fp16 x fp16, K-major
       constexpr uint32_t idesc_pv = idesc_f32acc(0, 0, 128, 256, 0, 1);    // P K-major, V MN-major
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
       bool ok = mbar_wait(&bar->q_full, 0, p.budget);
       if (!ok) report_error(p.err, kDevErrTimeout, 320, 0);
-      for (int i = 0; ok && i <= n_tiles; ++i) {
+      // QK^T runs two tiles ahead of PV: the softmax reads S(i+1) while it
+      // still works on tile i, so S(i+2) can be computed meanwhile.
+      for (int i = 0; ok && i < n_tiles + 2; ++i) {
         if (i < n_tiles) {
-          const int st = i & 1;
-          if (!mbar_wait(&bar->kv_full[st], (i >> 1) & 1, p.budget) ||
-              !mbar_wait(&bar->s_empty[st], ((i >> 1) & 1) ^ 1, p.budget)) {
+          const int st = i % kStages;
+          if (!mbar_wait(&bar->kv_full[st], (i / kStages) & 1, p.budget) ||
+              (i > 0 && !mbar_wait(&bar->s_empty, (i - 1) & 1, p.budget))) {
             report_error(p.err, kDevErrTimeout, 321, i);
             break;
           }
           tc_fence_after();
           const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
-          const uint32_t tS = tmem + 256 + st * 64;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma_bf16(tS, smem_desc(q_addr + c * 16384 + k * 32, 16, 1024, kSwizzle128B),
-                        smem_desc(kv_addr + c * 8192 + k * 32, 16, 1024, kSwizzle128B), idesc_qk,
-                        (c | k) ? 1u : 0u);
+              umma_f16_ts(tmem + TM_S, tmem + TM_Q + c * 32 + k * 8,
+                          smem_desc(kv_addr + c * 8192 + k * 32, 16, 1024, kSwizzle128B), idesc_qk,
+                          (c | k) ? 1u : 0u);
             }
           }
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
-            umma_bf16(tS, smem_desc(q_addr + Q_ROPE + k * 32, 16, 512, kSwizzle64B),
-                      smem_desc(kv_addr + KV_ROPE + k * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
+            umma_f16_ts(tmem + TM_S, tmem + TM_Q + 128 + k * 8,
+                        smem_desc(kv_addr + KV_ROPE + k * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
           }
-          umma_commit(&bar->s_full[st]);
+          umma_commit(&bar->s_full);
         }
-        if (i >= 1) {
-          const int j = i - 1;
-          const int st = j & 1;
-          if (!mbar_wait(&bar->p_full[st], (j >> 1) & 1, p.budget)) {
+        if (i >= 2) {
+          const int j = i - 2;
+          if (!mbar_wait(&bar->p_full, j & 1, p.budget)) {
             report_error(p.err, kDevErrTimeout, 322, j);
             break;
           }
           tc_fence_after();
+          const int st = j % kStages;
           const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
-          const uint32_t pb_addr = p_addr + st * P_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            umma_bf16(tmem, smem_desc(pb_addr + k * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(kv_addr + k * 2048, 8192, 1024, kSwizzle128B), idesc_pv, (j | k) ? 1u : 0u);
+            umma_f16_ts(tmem + TM_O, tmem + TM_P + k * 8,
+                        smem_desc(kv_addr + k * 2048, 8192, 1024, kSwizzle128B), idesc_pv, (j | k) ? 1u : 0u);
           }
-          umma_commit(&bar->pv_done[st]);
+          umma_commit(&bar->pv_done);
           umma_commit(&bar->kv_empty[st]);
         }
       }
     }
   } else {
-    // ------------------------------------------------ softmax warpgroup --
+    // -------------------------------------------------------------- softmax --
+    const int sw = static_cast<int>(warp) - C::SOFT0;   // 0..7
+    const int g = sw >> 2;                               // column half: keys [32g, 32g+32) of a tile
     const uint32_t quarter = warp & 3u;
     const int h = static_cast<int>(quarter * 32 + lane);
-    const uint32_t lane_addr = (quarter * 32u) << 16;
-    const uint32_t x_local = smem_u32(sX) + h * X_PITCH;
-    const uint32_t x_remote = mapa_shared(x_local, peer);
-    const uint32_t x_full_remote = mapa_shared(smem_u32(&bar->x_full), peer);
-    const uint32_t x_free_remote = mapa_shared(smem_u32(&bar->x_free), peer);
+    const uint32_t lane_base = tmem + ((quarter * 32u) << 16);
+    // partial-score blocks: this warp owns 2 KB (32 heads x 32 keys, fp16) per
+    // tile; the peer's warp with the same (g, quarter) fills the same block of
+    // our receive buffer.  16-byte unit q of lane l sits at unit q ^ ((l>>1)&3).
+    const int blk = g * 4 + static_cast<int>(quarter);
+    uint32_t uoff[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) uoff[q] = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+    const uint32_t stg_base = smem_u32(sm + OFF_STG) + blk * XBLK;
+    const uint32_t x_base = smem_u32(sm + OFF_X) + blk * XBLK;
+    const uint32_t x_base_remote = mapa_shared(x_base, peer);
+    const uint32_t x_full_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0]), peer),
+                                       mapa_shared(smem_u32(&bar->x_full[1]), peer)};
+    const uint32_t x_free_remote[2] = {mapa_shared(smem_u32(&bar->x_free[0]), peer),
+                                       mapa_shared(smem_u32(&bar->x_free[1]), peer)};
     const float NEG_INF = __int_as_float(0xff800000);
-    float m_run = NEG_INF;    // running max (log2 domain), refreshed lazily
-    float l_run = 0.f;
+    const float scale = p.scale_log2;
+    float m_run = NEG_INF;     // running max (log2 domain), refreshed lazily; identical in both halves
+    float l_run = 0.f;         // partial row sum over this half's columns
     bool ok = true;
-    // bounded wait whose outcome is the same for every lane of the warp
+    // bounded wait polled by lane 0; every lane gets the same outcome and is
+    // ordered after lane 0's acquire by the warp barrier
     auto wwait = [&](uint64_t* b_, uint32_t parity, bool cluster, uint32_t site, int info) -> bool {
-      const bool r = cluster ? mbar_wait_cluster(b_, parity, p.budget) : mbar_wait(b_, parity, p.budget);
-      if (!r) report_error(p.err, kDevErrTimeout, site, info);
-      return __all_sync(0xffffffffu, r);
+      int r = 1;
+      if (lane == 0) {
+        r = cluster ? mbar_wait_cluster(b_, parity, p.budget) : mbar_wait(b_, parity, p.budget);
+        if (!r) report_error(p.err, kDevErrTimeout, site, info);
+      }
+      r = __shfl_sync(0xffffffffu, r, 0);
+      __syncwarp();
+      return r != 0;
     };
+    // S(t) of head h, columns [32g, 32g+32), rounded to fp16 pairs (the peer
+    // receives exactly these values, so both CTAs add the same two numbers)
+    auto load_s = [&](int t, uint32_t (&pk)[16]) -> bool {
+      if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
+      tc_fence_after();
+      uint32_t sreg[32];
+      tmem_ld32(lane_base + TM_S + 32 * g, sreg);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->s_empty);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint32_t r;
+        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(sreg[2 * c + 1])),
+            "f"(__uint_as_float(sreg[2 * c])));
+        pk[c] = r;
+      }
+      return true;
+    };
+    // ship this warp's block of S(t) to the peer (one 2 KB bulk copy)
+    auto send = [&](int t, const uint32_t (&pk)[16]) -> bool {
+      const int xb = t & 1;
+      if (!wwait(&bar->x_free[xb], ((t >> 1) & 1) ^ 1, true, 331, t)) return false;
+      const uint32_t stg = stg_base + xb * XBUF;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + uoff[q]), "r"(pk[4 * q]),
+                     "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) bulk_copy_to_peer(x_base_remote + xb * XBUF, stg, XBLK, x_full_remote[xb]);
+      return true;
+    };
+
+    if (n_tiles > 0) {
+      // Q_r row h into TMEM: this half writes dims [144g, 144g+144) = columns [72g, 72g+72)
+      uint32_t qv[72];
+      const uint16_t* qrow = p.q + (static_cast<int64_t>(row) * H + h) * 576;
+#pragma unroll
+      for (int m = 0; m < 18; ++m) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (h < H) v = cvt_unit(__ldg(reinterpret_cast<const uint4*>(qrow + unit_dim(18 * g + m, rank))));
+        qv[4 * m + 0] = v.x;
+        qv[4 * m + 1] = v.y;
+        qv[4 * m + 2] = v.z;
+        qv[4 * m + 3] = v.w;
+      }
+      const uint32_t qaddr = lane_base + TM_Q + 72 * g;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t16[e] = qv[16 * c + e];
+        tmem_st16(qaddr + 16 * c, t16);
+      }
+      {
+        uint32_t t8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t8[e] = qv[64 + e];
+        tmem_st8(qaddr + 64, t8);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->q_full);
+    }
+
+    uint32_t cur[16], nxt[16];
+    if (n_tiles > 0) ok = load_s(0, cur) && send(0, cur);
     for (int i = 0; ok && i < n_tiles; ++i) {
-      const int st = i & 1;
-      // 1. this CTA's partial scores for head h
-      if (!wwait(&bar->s_full[st], (i >> 1) & 1, false, 330, i)) {
+      // 1. next tile's partial scores go out first, so the exchange overlaps this tile's work
+      if (i + 1 < n_tiles && !(load_s(i + 1, nxt) && send(i + 1, nxt))) {
+        ok = false;
+        break;
+      }
+      // 2. the peer's partial scores of tile i
+      const int xb = i & 1;
+      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xb], XBLK);
+      if (!wwait(&bar->x_full[xb], (i >> 1) & 1, true, 332, i)) {
+        ok = false;
+        break;
+      }
+      uint32_t xp[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(xp[4 * q]), "=r"(xp[4 * q + 1]), "=r"(xp[4 * q + 2]), "=r"(xp[4 * q + 3])
+                     : "r"(x_base + xb * XBUF + uoff[q])
+                     : "memory");
+      }
+      float sv[32];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&cur[c]));
+        const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&xp[c]));
+        sv[2 * c] = a.x + bb.x;
+        sv[2 * c + 1] = a.y + bb.y;
+      }
+      __syncwarp();
+      // the values are in registers: the peer may refill the buffer
+      if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote[xb]);
+      // 3. mask positions past the selection / padding
+      const uint32_t vbits = sValid[2 * i + g];
+      if (vbits != 0xffffffffu) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (!((vbits >> c) & 1u)) sv[c] = NEG_INF;
+      }
+      // 4. row max over all 64 columns (the other half through shared memory)
+      float pm = sv[0];
+#pragma unroll
+      for (int c = 1; c < 32; ++c) pm = fmaxf(pm, sv[c]);
+      float* red = sRed + (i & 1) * 256;     // double-buffered by tile parity
+      red[g * 128 + h] = pm;
+      mbar_arrive(&bar->red);
+      if (!wwait(&bar->red, i & 1, false, 336, i)) {
+        ok = false;
+        break;
+      }
+      const float mz = fmaxf(pm, red[(g ^ 1) * 128 + h]) * scale;
+      const float m_new = fmaxf(m_run, mz);
+      const bool grow = m_new > m_run + 8.0f;           // true on the first finite tile
+      float alpha = 1.f;
+      if (grow) {
+        alpha = fast_exp2(m_run - m_new);                // exp2(-inf) = 0
+        m_run = m_new;
+      }
+      const float m_ref = m_run == NEG_INF ? 0.f : m_run;
+      // 5. probabilities (fp16 pairs) and this half's row sum
+      uint32_t pk[16];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float pa = fast_exp2(fmaf(sv[2 * c], scale, -m_ref));
+        const float pb = fast_exp2(fmaf(sv[2 * c + 1], scale, -m_ref));
+        rs += pa + pb;
+        pk[c] = pack_half2(pa, pb);
+      }
+      l_run = l_run * alpha + rs;
+      // 6. PV(i-1) must be done before P and O are touched
+      if (i > 0 && !wwait(&bar->pv_done, (i - 1) & 1, false, 333, i)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sa[32], sb[32];
-      tmem_ld32(tmem + lane_addr + 256 + st * 64, sa);
-      tmem_ld32(tmem + lane_addr + 256 + st * 64 + 32, sb);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->s_empty[st]);
-      // 2. send them to the partner, 3. receive the partner's
-      if (!wwait(&bar->x_free, (i & 1) ^ 1, true, 331, i)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        st_cluster_v4(x_remote + q * 16, __uint_as_float(sa[4 * q]), __uint_as_float(sa[4 * q + 1]),
-                      __uint_as_float(sa[4 * q + 2]), __uint_as_float(sa[4 * q + 3]));
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        st_cluster_v4(x_remote + 128 + q * 16, __uint_as_float(sb[4 * q]), __uint_as_float(sb[4 * q + 1]),
-                      __uint_as_float(sb[4 * q + 2]), __uint_as_float(sb[4 * q + 3]));
-      }
-      mbar_arrive_remote(x_full_remote);
-      if (!wwait(&bar->x_full, i & 1, true, 332, i)) {
-        ok = false;
-        break;
-      }
-      const float4* xr = reinterpret_cast<const float4*>(reinterpret_cast<const uint8_t*>(sX) + h * X_PITCH);
-      const int* tidx = sIdx + i * kTileKeys;
-      float mz = NEG_INF;
-      // own + peer partial scores (the peer adds them in the other order: fp add
-      // commutes, so both CTAs hold bit-identical S), masked, in log2 units
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float4 x = xr[q];
-        uint32_t* src = q < 8 ? &sa[4 * q] : &sb[4 * (q - 8)];
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float zz = tidx[4 * q + e] >= 0 ? (__uint_as_float(src[e]) + xs[e]) * p.scale_log2 : NEG_INF;
-          src[e] = __float_as_uint(zz);
-          mz = fmaxf(mz, zz);
-        }
-      }
-      mbar_arrive_remote(x_free_remote);   // our buffer may be refilled by the peer
-      const float m_new = fmaxf(m_run, mz);
-      const bool grow = m_new > m_run + 8.0f;         // true on the first finite tile
-      float alpha = 1.f;
-      if (grow) {
-        alpha = fast_exp2(m_run - m_new);              // exp2(-inf) = 0
-        m_run = m_new;
-      }
-      const float m_ref = m_run == NEG_INF ? 0.f : m_run;
-      // P buffer (i & 1) is free once PV(i - 2) finished
-      if (i >= 2 && !wwait(&bar->pv_done[st], ((i - 2) >> 1) & 1, false, 333, i)) {
-        ok = false;
-        break;
-      }
-      // O may only be rescaled between PV(i - 1) and PV(i)
       if (i > 0 && __any_sync(0xffffffffu, grow)) {
-        if (!wwait(&bar->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, false, 334, i)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + c * 32, o);
+          const uint32_t oa = lane_base + TM_O + 128 * g + 32 * c;
+          tmem_ld32(oa, o);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tmem + lane_addr + c * 32, o);
+          tmem_st32(oa, o);
         }
-        tmem_st_wait();
       }
-      // P row h: fp16, 64 keys = 128 bytes, 128-byte swizzle
-      uint8_t* prow = sP + st * P_BYTES + h * 128;
-      float rs = 0.f;
-#pragma unroll
-      for (int cu = 0; cu < 8; ++cu) {
-        const uint32_t* src = cu < 4 ? &sa[8 * cu] : &sb[8 * (cu - 4)];
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pa = fast_exp2(__uint_as_float(src[2 * e]) - m_ref);
-          const float pb = fast_exp2(__uint_as_float(src[2 * e + 1]) - m_ref);
-          rs += pa + pb;
-          const __half2 hv = __floats2half2_rn(pa, pb);
-          w4[e] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        *reinterpret_cast<uint4*>(prow + ((cu ^ (h & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      l_run = l_run * alpha + rs;
-      fence_proxy_async_smem();
+      tmem_st16(lane_base + TM_P + 16 * g, pk);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar->p_full[st]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->p_full);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) cur[c] = nxt[c];
     }
+
     // ---- epilogue: O / l -> bf16 (or fp32 partial) ----
-    if (ok && n_tiles > 0 && !wwait(&bar->pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, false, 335, n_tiles)) {
-      ok = false;
-    }
+    if (ok && n_tiles > 0 && !wwait(&bar->pv_done, (n_tiles - 1) & 1, false, 335, n_tiles)) ok = false;
     tc_fence_after();
-    const float inv_l = (n_tiles > 0 && l_run > 0.f) ? 1.f / l_run : 0.f;
-    const float lse_val = (n_tiles > 0 && l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : NEG_INF;
+    float* lsum = sRed + 512;
+    lsum[g * 128 + h] = l_run;
+    mbar_arrive(&bar->red);
+    if (ok && !wwait(&bar->red, n_tiles & 1, false, 337, n_tiles)) ok = false;
+    const float l = lsum[h] + lsum[128 + h];            // same order in both halves
+    const bool any = n_tiles > 0 && l > 0.f;
+    const float inv_l = any ? 1.f / l : 0.f;
+    const float lse_val = any ? (m_run + __log2f(l)) * 0.69314718055994531f : NEG_INF;
     if (p.nsplit == 1) {
-      uint16_t* orow = p.out + (static_cast<int64_t>(row) * H + h) * 512 + rank * 256;
+      uint16_t* orow = p.out + (static_cast<int64_t>(row) * H + h) * 512 + rank * 256 + 128 * g;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         if (n_tiles > 0) {
-          tmem_ld32(tmem + lane_addr + c * 32, o);
+          tmem_ld32(lane_base + TM_O + 128 * g + 32 * c, o);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -472,15 +611,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
           }
         }
       }
-      if (rank == 0 && h < H && p.lse != nullptr) p.lse[static_cast<int64_t>(row) * H + h] = lse_val;
+      if (rank == 0 && g == 0 && h < H && p.lse != nullptr) p.lse[static_cast<int64_t>(row) * H + h] = lse_val;
     } else {
       const int64_t prow_i = (static_cast<int64_t>(row) * p.nsplit + split) * 128 + h;
-      float* orow = p.part_o + prow_i * 512 + rank * 256;
+      float* orow = p.part_o + prow_i * 512 + rank * 256 + 128 * g;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         if (n_tiles > 0) {
-          tmem_ld32(tmem + lane_addr + c * 32, o);
+          tmem_ld32(lane_base + TM_O + 128 * g + 32 * c, o);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -493,16 +632,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1) sparse_
                           __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
         }
       }
-      if (rank == 0) p.part_lse[prow_i] = lse_val;
+      if (rank == 0 && g == 0) p.part_lse[prow_i] = lse_val;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   cluster_sync();          // the peer no longer touches our shared memory
-  if (warp == kMmaWarp) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// bf16 -> fp16 copy of the latent cache (saturating, exact in the normal range).
+__global__ void __launch_bounds__(256) latent_to_fp16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                             int64_t n_units) {
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    dst[u] = cvt_unit(__ldg(&src[u]));
   }
 }
 
@@ -543,10 +691,20 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   }
 }
 
+template <bool TMA>
+cudaError_t launch_variant(dim3 grid, const MlaParams& p, const CUtensorMap& ml, const CUtensorMap& mr,
+                           cudaStream_t stream) {
+  cudaError_t e =
+      cudaFuncSetAttribute(sparse_mla_kernel<TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  sparse_mla_kernel<TMA><<<grid, Cfg<TMA>::THREADS, kSmem, stream>>>(p, ml, mr);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int mla_num_splits(int total_q, int max_q_per_seq, int num_seqs, int k_sel) {
-  // fill ~2 waves of CTA pairs (74 pairs per wave on 148 SMs); keep >= 4 tiles per split
+  // fill the 74 CTA pairs of one wave about twice; keep >= 4 tiles per split
   (void)max_q_per_seq;
   (void)num_seqs;
   const int max_tiles = (k_sel + kTileKeys - 1) / kTileKeys;
@@ -560,12 +718,30 @@ int mla_keys_per_split(int k_sel, int nsplit) {
   return ((tiles + nsplit - 1) / nsplit) * kTileKeys;
 }
 
+bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_sel) {
+  // the copy reads and writes every cache row once; worth it when each row is
+  // gathered about 8 times or more
+  const int64_t gathers = static_cast<int64_t>(total_q) * (k_sel < max_kv_len ? k_sel : max_kv_len);
+  return gathers >= 8 * total_keys;
+}
+
 size_t mla_smem_bytes() { return kSmem; }
 
 cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (e != cudaSuccess) return e;
-  sparse_mla_kernel<<<grid, kThreads, kSmem, stream>>>(p);
+  CUtensorMap unused;
+  std::memset(&unused, 0, sizeof(unused));
+  return launch_variant<false>(grid, p, unused, unused, stream);
+}
+
+cudaError_t launch_sparse_mla_tma(dim3 grid, const MlaParams& p, const CUtensorMap& map_lat,
+                                  const CUtensorMap& map_rope, cudaStream_t stream) {
+  return launch_variant<true>(grid, p, map_lat, map_rope, stream);
+}
+
+cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream) {
+  const int64_t units = n_elems / 8;
+  latent_to_fp16_kernel<<<148 * 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(src),
+                                                     reinterpret_cast<uint4*>(dst), units);
   return cudaGetLastError();
 }
 

@@ -52,6 +52,7 @@ def test_tiny_prefill_512_every_row():
     ([4000, 3100, 5000, 257], [1, 1, 1, 1], 2048, 128),            # decode: 1 token, split MLA
     ([6000, 4100, 2049, 3000], [2, 2, 2, 2], 2048, 128),           # speculative pairs
     ([700, 900], [5, 4], 512, 32),                                 # 4-token indexer blocks
+    ([2100 + 37 * i for i in range(40)], [1] * 40, 2048, 128),      # decode split into 4 x 8 tiles
     ([128, 256, 384], [128, 17, 256], 64, 16),                     # exact tile multiples
 ])
 def test_ragged_batches(kv, q, k_sel, H):
