@@ -162,9 +162,11 @@ dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int
   p.ld = ld;
   p.k_sel = k_sel;
   p.idx = idx;
+  p.total_q = b->total_q;
+  p.num_seqs = b->num_seqs;
   p.err = err;
-  const dim3 grid(b->max_q_per_seq, b->num_seqs);
-  return dsa::launch_topk(b->max_kv_len, grid, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  p.budget = wait_budget();
+  return dsa::launch_topk(b->max_kv_len, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const void* kv, const int32_t* idx,

@@ -40,10 +40,13 @@ struct TopkParams {
   int64_t ld;
   int32_t k_sel;
   int32_t* idx;           // [total_q, k_sel]
+  int32_t total_q;
+  int32_t num_seqs;
   uint32_t* err;
+  long long budget;       // clock64 cycles a bulk-copy wait may take
 };
 
-cudaError_t launch_topk(int max_kv_len, dim3 grid, const TopkParams& p, cudaStream_t stream);
+cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream);
 
 // ------------------------------------------------------------- sparse MLA --
 struct MlaParams {

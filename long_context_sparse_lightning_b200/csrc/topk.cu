@@ -1,33 +1,52 @@
-// Per-query top-k over the causal prefix of each score row: radix select on
-// order-preserving uint32 keys of the fp32 scores, then an ordered compaction.
+// Per-query top-k over the causal prefix of each score row.
 //
 // Eq. (2) of "详解DSA": S_t = { s : I[t, s] in Top-k(I[t, :]) } over s <= t; a
 // row with at most k positions keeps them all ("详解DSA", prefill analysis).
 // "DeepSeek V3.2 稀疏注意力" (top-k as the algorithm/kernel interface) asks for
 // a selection kernel rather than a generic sort, with the tie and padding rules
-// defined; here: higher score first, ties broken by the lower position, output
-// = the selected set in ascending position order within each of the two
-// groups (strictly above the threshold, then threshold ties), -1 padding.
+// defined; here: higher score first, ties broken by the lower position (scores
+// compare as floats, so -0 and +0 tie), output = the selected positions in
+// ascending order, -1 padding.
 //
-// One CTA per query row.  Rows up to BLOCK*32 positions keep their keys in
-// registers (32 per thread, loaded once with 16-byte loads); longer rows are
-// re-streamed from global memory (L2) on every pass.  Three histogram passes
-// over 11/11/10-bit digits (2048 shared-memory bins, warp-aggregated atomics)
-// locate the exact 32-bit threshold key T and how many of the T-valued
-// positions are needed; a final pass writes the positions in index order using
-// block-wide prefix sums.
+// Selection is one histogram pass in value space, not a digit-by-digit radix
+// select: the row's finite range [min, max] is cut into 2048 equal-width bins
+// (a monotone map of the value, so bins are ordered like the scores), a
+// shared-memory histogram locates the bin b* that holds the k-th largest score,
+// every position above b* is selected, and the few positions inside b* (tens
+// on indexer score rows) are ranked against each other exactly.  Equal-width
+// value bins spread the bulk of a score row over hundreds of bins, where the
+// top bits of the float encoding would pile it into a handful and serialise
+// the shared-memory atomics.  Rows whose boundary bin holds more than
+// kCandCap positions, or that contain a non-finite score, take an exact
+// 32-bit radix select instead (11/11/10-bit digits on order-preserving keys).
+//
+// Rows of up to 32768 positions run in a persistent kernel: each CTA keeps the
+// current row in registers (up to 64 scores per thread) while the bulk-copy
+// engine streams its next row into shared memory.  Longer rows run one CTA
+// per row and re-read the row from global memory (L2) on every pass.
+#include <algorithm>
+#include <cfloat>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kEPT = 32;             // keys per thread in the register path
 constexpr int kBins = 2048;
+constexpr int kCandCap = 512;     // boundary-bin positions ranked pairwise
+constexpr int kSegChunks = 16;    // chunks per compaction segment: 16 x 4 flags per thread
 
 __device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;     // -0 ties with +0, as in a float comparison
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
 // Exclusive prefix sum over the block, in thread order; also returns the total.
@@ -59,80 +78,299 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return before + x - v;
 }
 
-template <int BLOCK, bool IN_REGS>
-__global__ void __launch_bounds__(BLOCK) topk_kernel(const TopkParams p) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t s_warp[32];
-  __shared__ uint32_t s_digit, s_above;
-  const int k_out = p.k_sel;
+template <int BLOCK>
+struct TopkShared {
+  static constexpr int NW = BLOCK / 32;
+  uint32_t hist[kBins];
+  float cand_v[kCandCap];
+  int32_t cand_p[kCandCap];
+  uint8_t cand_sel[kCandCap];
+  uint32_t tab[kSegChunks * NW];
+  uint32_t s_warp[32];
+  float s_max[32], s_min[32];
+  uint32_t s_bstar, s_above, s_cnt, s_ncand, s_total, s_digit;
+  alignas(8) uint64_t bar;
+};
 
-  if (error_pending(p.err)) return;
-  const int b = blockIdx.y;
-  const int i = blockIdx.x;
-  const int q0 = __ldg(&p.cu_q[b]);
-  const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
-  if (i >= q_len) return;
-  const int kv = __ldg(&p.kv_len[b]);
-  const int r = q0 + i;
+// Sequence of query row r (binary search over cu_q) and its causal length n.
+__device__ __forceinline__ bool row_info(const TopkParams& p, int r, int& n) {
+  int lo = 0, hi = p.num_seqs;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(&p.cu_q[mid]) <= r) lo = mid;
+    else hi = mid;
+  }
+  const int q0 = __ldg(&p.cu_q[lo]);
+  const int q_len = __ldg(&p.cu_q[lo + 1]) - q0;
+  const int kv = __ldg(&p.kv_len[lo]);
+  const int i = r - q0;
   const int t = kv - q_len + i;
-  const int k = p.k_sel;
-  int32_t* out = p.idx + static_cast<int64_t>(r) * k;
-  if (t < 0 || kv > p.ld) {
-    if (threadIdx.x == 0) report_error(p.err, kDevErrBounds, 201, r);
-    return;
-  }
-  const int n = t + 1;
-  if (n <= k) {
-    for (int j = threadIdx.x; j < k; j += BLOCK) out[j] = j < n ? j : -1;
-    return;
-  }
-  const float* row = p.scores + static_cast<int64_t>(r) * p.ld;
-  const int tid = threadIdx.x;
-  const int n_vec = (n + 3) >> 2;                         // float4 vectors covering the row
-  const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;       // vectors per thread (register path: <= kEPT/4)
+  if (i < 0 || i >= q_len || t < 0 || kv > p.ld) return false;
+  n = t + 1;
+  return true;
+}
 
-  uint32_t keys[IN_REGS ? kEPT : 1];
-  if constexpr (IN_REGS) {
+// Selects the top k of one row with n > k positions and writes them to `out`.
+// get4(v) returns the float4 of vector v*BLOCK + tid (positions 4 * that ..+3).
+// EPT > 0: the row is held in registers, EPT positions per thread, and every
+// chunk loop is unrolled; EPT == 0: get4 reads memory, loops stay rolled.
+// Calls fn(v) for v in [v0, v1): unrolled over the EPT/4 register chunks when
+// EPT > 0, a rolled loop otherwise.
+template <int EPT, typename Fn>
+__device__ __forceinline__ void for_range(int v0, int v1, Fn&& fn) {
+  if constexpr (EPT > 0) {
 #pragma unroll
-    for (int v = 0; v < kEPT / 4; ++v) {
-      const int vec = v * BLOCK + tid;
-      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (vec < n_vec) f = __ldg(reinterpret_cast<const float4*>(row) + vec);
-      keys[4 * v + 0] = order_key(f.x);
-      keys[4 * v + 1] = order_key(f.y);
-      keys[4 * v + 2] = order_key(f.z);
-      keys[4 * v + 3] = order_key(f.w);
-    }
-  }
-  // key of component c of this thread's vector in chunk v (position (v*BLOCK+tid)*4+c)
-  auto load4 = [&](int v, uint32_t (&k4)[4]) {
-    if constexpr (IN_REGS) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) k4[c] = keys[4 * v + c];
-    } else {
-      const int vec = v * BLOCK + tid;
-      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (vec < n_vec) f = __ldg(reinterpret_cast<const float4*>(row) + vec);
-      k4[0] = order_key(f.x);
-      k4[1] = order_key(f.y);
-      k4[2] = order_key(f.z);
-      k4[3] = order_key(f.w);
-    }
-  };
-
-  // visit this thread's vectors in position order (unrolled when keys live in registers)
-  auto for_chunks = [&](auto&& fn) {
-    if constexpr (IN_REGS) {
-#pragma unroll
-      for (int v = 0; v < kEPT / 4; ++v)
-        if (v < n_chunks) fn(v);
-    } else {
+    for (int v = 0; v < EPT / 4; ++v)
+      if (v >= v0 && v < v1) fn(v);
+  } else {
 #pragma unroll 1
-      for (int v = 0; v < n_chunks; ++v) fn(v);
+    for (int v = v0; v < v1; ++v) fn(v);
+  }
+}
+
+// max / min that return NaN when either input is NaN
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Value-bin selection.  Returns false, having written nothing, when the row
+// holds a non-finite score or its boundary bin holds more than kCandCap
+// positions; the caller then runs select_radix.
+template <int BLOCK, int EPT, typename Get4>
+__device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, int n, int n_chunks, int k,
+                                            int32_t* __restrict__ out) {
+  constexpr int NW = BLOCK / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t FULL = 0xffffffffu;
+  auto pos_of = [&](int v, int c) { return (v * BLOCK + tid) * 4 + c; };
+
+  // ---- range of the row (NaN-propagating, so any NaN or inf shows) ----
+  float mx = -FLT_MAX, mn = FLT_MAX;
+  for_range<EPT>(0, n_chunks, [&](int v) {
+    const float4 f = get4(v);
+    const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (pos_of(v, c) < n) {
+        mx = max_nan(mx, e[c]);
+        mn = min_nan(mn, e[c]);
+      }
     }
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = max_nan(mx, __shfl_xor_sync(FULL, mx, o));
+    mn = min_nan(mn, __shfl_xor_sync(FULL, mn, o));
+  }
+  if (lane == 0) {
+    sh.s_max[warp] = mx;
+    sh.s_min[warp] = mn;
+  }
+  for (int j = tid; j < kBins; j += BLOCK) sh.hist[j] = 0u;
+  if (tid == 0) sh.s_ncand = 0u;
+  __syncthreads();
+  mx = sh.s_max[0];
+  mn = sh.s_min[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    mx = max_nan(mx, sh.s_max[w]);
+    mn = min_nan(mn, sh.s_min[w]);
+  }
+  if (!(fabsf(mx) <= FLT_MAX && fabsf(mn) <= FLT_MAX)) return false;   // uniform
+
+  // Bin of a score: the integer part of 2^23 + (x - mn) * 2048 / (mx - mn),
+  // read from the float's bits and clamped to [0, 2047].  One rounding (fma)
+  // of a function increasing in x, so the map is monotone: bins are ordered
+  // like the scores.  (The candidates inside b* are then ranked exactly, so
+  // rounding only moves positions between neighbouring bins.)
+  const float scale = static_cast<float>(kBins) / (mx - mn);
+  const float off = 8388608.0f - mn * scale;
+  auto bin_of = [&](float x) -> int {
+    const int b = static_cast<int>(__float_as_uint(__fmaf_rn(x, scale, off))) - 0x4B000000;
+    return min(max(b, 0), kBins - 1);
   };
 
-  // ---- radix select: 11 + 11 + 10 bits from the top ----
+  // ---- histogram ----
+  for_range<EPT>(0, n_chunks, [&](int v) {
+    const float4 f = get4(v);
+    const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (pos_of(v, c) < n) atomicAdd(&sh.hist[bin_of(e[c])], 1u);
+  });
+  __syncthreads();
+  // ---- bin b* with count(bins above) < k <= count(bins at or above) ----
+  {
+    constexpr int BPT = kBins / BLOCK;
+    uint32_t local[BPT];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      local[j] = sh.hist[kBins - 1 - (tid * BPT + j)];
+      sum += local[j];
+    }
+    uint32_t total;
+    uint32_t above = block_excl_scan<BLOCK>(sum, sh.s_warp, total);
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (above < static_cast<uint32_t>(k) && above + local[j] >= static_cast<uint32_t>(k)) {
+        sh.s_bstar = static_cast<uint32_t>(kBins - 1 - (tid * BPT + j));
+        sh.s_above = above;
+        sh.s_cnt = local[j];
+      }
+      above += local[j];
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(sh.s_bstar);
+  const uint32_t rem = static_cast<uint32_t>(k) - sh.s_above;
+  if (sh.s_cnt > static_cast<uint32_t>(kCandCap)) return false;             // uniform
+
+  // ---- classify: above b* (selected) / inside b* (ranked); collect b* ----
+  // masks hold one bit per position of a segment of kSegChunks chunks
+  auto classify = [&](int seg0, int seg1, bool collect, uint64_t& sel, uint64_t& inb) {
+    sel = 0;
+    inb = 0;
+    for_range<EPT>(seg0, seg1, [&](int v) {
+      const float4 f = get4(v);
+      const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int pos = pos_of(v, c);
+        const int b = pos < n ? bin_of(e[c]) : -1;
+        const uint64_t bit = uint64_t(1) << (4 * (v - seg0) + c);
+        if (b > bstar) sel |= bit;
+        const bool is = b == bstar;
+        if (is) inb |= bit;
+        if (collect) {
+          const uint32_t m = __ballot_sync(FULL, is);
+          if (m != 0u) {
+            const int leader = __ffs(m) - 1;
+            uint32_t base = 0;
+            if (lane == leader) base = atomicAdd(&sh.s_ncand, static_cast<uint32_t>(__popc(m)));
+            base = __shfl_sync(FULL, base, leader);
+            const uint32_t slot = base + __popc(m & lanemask_lt());
+            if (is && slot < static_cast<uint32_t>(kCandCap)) {
+              sh.cand_v[slot] = e[c];
+              sh.cand_p[slot] = pos;
+            }
+          }
+        }
+      }
+    });
+  };
+  // register rows fit one segment (EPT / 4 <= kSegChunks): classify once
+  static_assert(EPT / 4 <= kSegChunks, "a register row must fit one segment");
+  const bool one_seg = EPT > 0 || n_chunks <= kSegChunks;
+  uint64_t sel = 0, inb = 0;
+  if (one_seg) {
+    classify(0, n_chunks, true, sel, inb);
+  } else {
+    for (int seg0 = 0; seg0 < n_chunks; seg0 += kSegChunks)
+      classify(seg0, min(seg0 + kSegChunks, n_chunks), true, sel, inb);
+  }
+  __syncthreads();
+  // rank each b* position (higher score first, then lower position); the
+  // first `rem` are selected
+  const uint32_t ncand = min(sh.s_ncand, static_cast<uint32_t>(kCandCap));
+  for (uint32_t i = tid; i < ncand; i += BLOCK) {
+    const float x = sh.cand_v[i];
+    const int pos = sh.cand_p[i];
+    uint32_t rank = 0;
+    for (uint32_t j = 0; j < ncand; ++j) {
+      const float y = sh.cand_v[j];
+      rank += (y > x) || (y == x && sh.cand_p[j] < pos);
+    }
+    sh.cand_sel[i] = rank < rem;
+  }
+  __syncthreads();
+
+  // ---- ordered compaction, segment by segment ----
+  uint32_t base = 0;
+#pragma unroll 1
+  for (int seg0 = 0; seg0 < n_chunks; seg0 += kSegChunks) {
+    const int seg1 = min(seg0 + kSegChunks, n_chunks);
+    if (!one_seg) classify(seg0, seg1, false, sel, inb);
+#pragma unroll 1
+    while (inb != 0) {               // this thread's b* positions: look up their verdict
+      const int bit = __ffsll(static_cast<long long>(inb)) - 1;
+      inb &= inb - 1;
+      const int pos = ((seg0 + (bit >> 2)) * BLOCK + tid) * 4 + (bit & 3);
+      for (uint32_t j = 0; j < ncand; ++j)
+        if (sh.cand_p[j] == pos && sh.cand_sel[j]) sel |= uint64_t(1) << bit;
+    }
+    for_range<EPT>(seg0, seg1, [&](int v) {
+      const uint32_t fl = static_cast<uint32_t>(sel >> (4 * (v - seg0))) & 15u;
+      const uint32_t tot = __reduce_add_sync(FULL, static_cast<uint32_t>(__popc(fl)));
+      if (lane == 0) sh.tab[(v - seg0) * NW + warp] = tot;
+    });
+    __syncthreads();
+    if (warp == 0) {
+      constexpr int PER = kSegChunks * NW / 32;
+      const int n_ent = (seg1 - seg0) * NW;
+      uint32_t loc[PER];
+      uint32_t s = 0;
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int e = lane * PER + j;
+        loc[j] = e < n_ent ? sh.tab[e] : 0u;
+        s += loc[j];
+      }
+      uint32_t x = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+      }
+      uint32_t run = base + x - s;
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int e = lane * PER + j;
+        if (e < n_ent) sh.tab[e] = run;
+        run += loc[j];
+      }
+      if (lane == 31) sh.s_total = base + x;
+    }
+    __syncthreads();
+    const uint32_t lt = lanemask_lt();
+    for_range<EPT>(seg0, seg1, [&](int v) {
+      const uint32_t fl = static_cast<uint32_t>(sel >> (4 * (v - seg0))) & 15u;
+      // selected positions of lower lanes in this chunk, then lower components
+      uint32_t o = sh.tab[(v - seg0) * NW + warp];
+      o += __popc(__ballot_sync(FULL, fl & 1u) & lt) + __popc(__ballot_sync(FULL, fl & 2u) & lt) +
+           __popc(__ballot_sync(FULL, fl & 4u) & lt) + __popc(__ballot_sync(FULL, fl & 8u) & lt);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if ((fl >> c) & 1u) {
+          if (o < static_cast<uint32_t>(k)) out[o] = pos_of(v, c);
+          ++o;
+        }
+      }
+    });
+    base = sh.s_total;
+    __syncthreads();
+  }
+  return true;
+}
+
+// Exact radix select on order-preserving keys (11/11/10-bit digits,
+// warp-aggregated histogram updates), for rows select_fast declines: finds the
+// threshold key T and how many T-valued positions are needed, then writes the
+// selected positions in ascending order.
+template <int BLOCK, typename Get4>
+__device__ __noinline__ void select_radix(TopkShared<BLOCK>& sh, Get4 get4, int n, int n_chunks, int k,
+                                          int32_t* __restrict__ out) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t FULL = 0xffffffffu;
+  auto for_chunks = [&](auto&& fn) { for_range<0>(0, n_chunks, fn); };
+  auto pos_of = [&](int v, int c) { return (v * BLOCK + tid) * 4 + c; };
   uint32_t prefix = 0;
   uint32_t remaining = static_cast<uint32_t>(k);
 #pragma unroll 1
@@ -140,83 +378,83 @@ __global__ void __launch_bounds__(BLOCK) topk_kernel(const TopkParams p) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int width = pass == 2 ? 10 : 11;
     const uint32_t mask = (1u << width) - 1u;
-    for (int j = tid; j < kBins; j += BLOCK) hist[j] = 0u;
+    for (int j = tid; j < kBins; j += BLOCK) sh.hist[j] = 0u;
     __syncthreads();
-    const int upper = shift + width;   // bits above the current digit must equal prefix
+    const int upper = shift + width;
     for_chunks([&](int v) {
-      uint32_t k4[4];
-      load4(v, k4);
+      const float4 f = get4(v);
+      const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int pos = (v * BLOCK + tid) * 4 + c;
-        const bool match = pos < n && (upper >= 32 || (k4[c] >> upper) == prefix);
-        const uint32_t digit = (k4[c] >> shift) & mask;
-        const uint32_t active = __ballot_sync(0xffffffffu, match);
+        const uint32_t key = order_key(e[c]);
+        const bool match = pos_of(v, c) < n && (upper >= 32 || (key >> upper) == prefix);
+        const uint32_t digit = (key >> shift) & mask;
+        const uint32_t active = __ballot_sync(FULL, match);
         if (match) {
           const uint32_t peers = __match_any_sync(active, digit);
-          if ((__ffs(peers) - 1) == static_cast<int>(threadIdx.x & 31)) atomicAdd(&hist[digit], __popc(peers));
+          if ((__ffs(peers) - 1) == lane) atomicAdd(&sh.hist[digit], static_cast<uint32_t>(__popc(peers)));
         }
       }
     });
     __syncthreads();
-    // find the digit d with count(> d) < remaining <= count(>= d), scanning from the top bin
-    constexpr int BPT = kBins / BLOCK;        // bins per thread (>= 2)
+    constexpr int BPT = kBins / BLOCK;
     uint32_t local[BPT];
     uint32_t sum = 0;
 #pragma unroll
     for (int j = 0; j < BPT; ++j) {
-      local[j] = hist[kBins - 1 - (tid * BPT + j)];
+      local[j] = sh.hist[kBins - 1 - (tid * BPT + j)];
       sum += local[j];
     }
     if (tid == 0) {
-      s_digit = 0u;
-      s_above = 0u;
+      sh.s_digit = 0u;
+      sh.s_above = 0u;
     }
     uint32_t total;
-    uint32_t above = block_excl_scan<BLOCK>(sum, s_warp, total);
+    uint32_t above = block_excl_scan<BLOCK>(sum, sh.s_warp, total);
 #pragma unroll
     for (int j = 0; j < BPT; ++j) {
       if (above < remaining && above + local[j] >= remaining) {
-        s_digit = static_cast<uint32_t>(kBins - 1 - (tid * BPT + j));
-        s_above = above;
+        sh.s_digit = static_cast<uint32_t>(kBins - 1 - (tid * BPT + j));
+        sh.s_above = above;
       }
       above += local[j];
     }
     __syncthreads();
-    prefix = (prefix << width) | s_digit;
-    remaining -= s_above;
+    prefix = (prefix << width) | sh.s_digit;
+    remaining -= sh.s_above;
     __syncthreads();
   }
-  const uint32_t T = prefix;                 // exact threshold key
-  const uint32_t n_gt = static_cast<uint32_t>(k) - remaining;   // positions strictly above T
-
-  // ---- ordered compaction ----
+  const uint32_t T = prefix;
+  // a position's output slot = positions selected before it: (#above T before)
+  // + min(#ties before, remaining); the first `remaining` ties are selected
   uint32_t base_gt = 0, base_eq = 0;
   for_chunks([&](int v) {
-    uint32_t k4[4];
-    load4(v, k4);
+    const float4 f = get4(v);
+    const float e[4] = {f.x, f.y, f.z, f.w};
     uint32_t gt = 0, eq = 0;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int pos = (v * BLOCK + tid) * 4 + c;
-      if (pos < n) {
-        gt += k4[c] > T;
-        eq += k4[c] == T;
+      if (pos_of(v, c) < n) {
+        const uint32_t key = order_key(e[c]);
+        gt += key > T;
+        eq += key == T;
       }
     }
     uint32_t total;
-    const uint32_t off = block_excl_scan<BLOCK>((gt << 16) | eq, s_warp, total);
+    const uint32_t off = block_excl_scan<BLOCK>((gt << 16) | eq, sh.s_warp, total);
     uint32_t o_gt = base_gt + (off >> 16);
     uint32_t o_eq = base_eq + (off & 0xFFFFu);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int pos = (v * BLOCK + tid) * 4 + c;
+      const int pos = pos_of(v, c);
       if (pos < n) {
-        if (k4[c] > T) {
-          if (o_gt < static_cast<uint32_t>(k_out)) out[o_gt] = pos;
+        const uint32_t key = order_key(e[c]);
+        if (key > T) {
+          const uint32_t o = o_gt + min(o_eq, remaining);
+          if (o < static_cast<uint32_t>(k)) out[o] = pos;
           ++o_gt;
-        } else if (k4[c] == T) {
-          if (o_eq < remaining && n_gt + o_eq < static_cast<uint32_t>(k_out)) out[n_gt + o_eq] = pos;
+        } else if (key == T) {
+          if (o_eq < remaining && o_gt + o_eq < static_cast<uint32_t>(k)) out[o_gt + o_eq] = pos;
           ++o_eq;
         }
       }
@@ -226,18 +464,179 @@ __global__ void __launch_bounds__(BLOCK) topk_kernel(const TopkParams p) {
   });
 }
 
-template <int BLOCK, bool IN_REGS>
-cudaError_t launch_cfg(dim3 grid, const TopkParams& p, cudaStream_t stream) {
-  topk_kernel<BLOCK, IN_REGS><<<grid, BLOCK, 0, stream>>>(p);
+// get4 over a row in global memory (read through L1 / L2).
+template <int BLOCK>
+struct GlobalRow {
+  const float4* row4;
+  int n_vec;
+  __device__ __forceinline__ float4 operator()(int v) const {
+    const int vec = v * BLOCK + static_cast<int>(threadIdx.x);
+    return vec < n_vec ? __ldg(row4 + vec) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+};
+
+__device__ __forceinline__ void fill_short_row(int32_t* out, int n, int k, int block) {
+  for (int j = threadIdx.x; j < k; j += block) out[j] = j < n ? j : -1;
+}
+
+// Global -> shared bulk copy of one row (positions 0 .. n-1, rounded up to a
+// whole float4; the row stride is a multiple of 4 floats and >= that).
+__device__ __forceinline__ void issue_row_copy(float* buf, const float* row, int n, uint64_t* bar) {
+  const uint32_t bytes = static_cast<uint32_t>((n + 3) & ~3) * 4u;
+  fence_proxy_async_smem();   // earlier generic reads of the buffer precede the async writes
+  mbar_arrive_expect_tx(bar, bytes);
+  constexpr uint32_t kPiece = 32768;
+  for (uint32_t off = 0; off < bytes; off += kPiece) {
+    const uint32_t sz = min(kPiece, bytes - off);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(reinterpret_cast<const uint8_t*>(buf) + off)),
+        "l"(reinterpret_cast<const uint8_t*>(row) + off), "r"(sz), "r"(smem_u32(bar))
+        : "memory");
+  }
+}
+
+template <int BLOCK, int EPT>
+constexpr size_t reg_smem_bytes() {
+  return ((sizeof(TopkShared<BLOCK>) + 127) / 128) * 128 + static_cast<size_t>(BLOCK) * EPT * sizeof(float);
+}
+
+// Persistent kernel for rows of up to BLOCK*EPT positions: the row being
+// selected lives in registers, the CTA's next row is bulk-copied into shared
+// memory meanwhile.
+template <int BLOCK, int EPT, int MIN_CTAS>
+__global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkParams p) {
+  extern __shared__ __align__(128) uint8_t dyn[];
+  auto& sh = *reinterpret_cast<TopkShared<BLOCK>*>(dyn);
+  float* buf = reinterpret_cast<float*>(dyn + ((sizeof(TopkShared<BLOCK>) + 127) / 128) * 128);
+  constexpr int CAP = BLOCK * EPT;
+  const int k = p.k_sel;
+  const int tid = threadIdx.x;
+  const int G = gridDim.x;
+
+  if (error_pending(p.err)) return;
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto needs_copy = [&](int r, int& n) { return r < p.total_q && row_info(p, r, n) && n > k && n <= CAP; };
+  const float* scores = p.scores;
+  uint32_t phase = 0;
+  bool pending = false;
+  {
+    int n0;
+    if (needs_copy(blockIdx.x, n0)) {
+      if (tid == 0) issue_row_copy(buf, scores + static_cast<int64_t>(blockIdx.x) * p.ld, n0, &sh.bar);
+      pending = true;
+    }
+  }
+#pragma unroll 1
+  for (int r = blockIdx.x; r < p.total_q; r += G) {
+    int n = 0;
+    int32_t* out = p.idx + static_cast<int64_t>(r) * k;
+    if (!row_info(p, r, n) || n > CAP) {
+      if (tid == 0) report_error(p.err, kDevErrBounds, 201, r);
+      continue;
+    }
+    if (n <= k) {
+      fill_short_row(out, n, k, BLOCK);
+      continue;
+    }
+    if (!pending && tid == 0) issue_row_copy(buf, scores + static_cast<int64_t>(r) * p.ld, n, &sh.bar);
+    pending = false;
+    const bool ok = mbar_wait(&sh.bar, phase, p.budget);
+    phase ^= 1u;
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0) report_error(p.err, kDevErrTimeout, 202, r);
+      break;
+    }
+    const int n_vec = (n + 3) >> 2;
+    const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
+    float x[EPT];
+    const float4* b4 = reinterpret_cast<const float4*>(buf);
+#pragma unroll
+    for (int v = 0; v < EPT / 4; ++v) {
+      const int vec = v * BLOCK + tid;
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (vec < n_vec) f = b4[vec];
+      x[4 * v + 0] = f.x;
+      x[4 * v + 1] = f.y;
+      x[4 * v + 2] = f.z;
+      x[4 * v + 3] = f.w;
+    }
+    __syncthreads();   // the buffer is free: start the next row's copy
+    {
+      int nn;
+      if (needs_copy(r + G, nn)) {
+        if (tid == 0) issue_row_copy(buf, scores + static_cast<int64_t>(r + G) * p.ld, nn, &sh.bar);
+        pending = true;
+      }
+    }
+    auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
+    if (!select_fast<BLOCK, EPT>(sh, get4, n, n_chunks, k, out)) {
+      const GlobalRow<BLOCK> g{reinterpret_cast<const float4*>(scores + static_cast<int64_t>(r) * p.ld), n_vec};
+      select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
+    }
+  }
+}
+
+// One CTA per row for rows longer than the register path holds.
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) {
+  __shared__ TopkShared<BLOCK> sh;
+  const int k = p.k_sel;
+  const int r = blockIdx.x;
+  if (error_pending(p.err)) return;
+  int n = 0;
+  if (!row_info(p, r, n)) {
+    if (threadIdx.x == 0) report_error(p.err, kDevErrBounds, 201, r);
+    return;
+  }
+  int32_t* out = p.idx + static_cast<int64_t>(r) * k;
+  if (n <= k) {
+    fill_short_row(out, n, k, BLOCK);
+    return;
+  }
+  const float4* row4 = reinterpret_cast<const float4*>(p.scores + static_cast<int64_t>(r) * p.ld);
+  const int n_vec = (n + 3) >> 2;
+  const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
+  const GlobalRow<BLOCK> g{row4, n_vec};
+  if (!select_fast<BLOCK, 0>(sh, g, n, n_chunks, k, out)) select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
+template <int BLOCK, int EPT, int MIN_CTAS>
+cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
+  constexpr size_t smem = reg_smem_bytes<BLOCK, EPT>();
+  cudaError_t e = cudaFuncSetAttribute(topk_reg_kernel<BLOCK, EPT, MIN_CTAS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(p.total_q, sm_count() * MIN_CTAS);
+  topk_reg_kernel<BLOCK, EPT, MIN_CTAS><<<grid, BLOCK, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_topk(int max_kv_len, dim3 grid, const TopkParams& p, cudaStream_t stream) {
-  if (max_kv_len <= 256 * kEPT) return launch_cfg<256, true>(grid, p, stream);
-  if (max_kv_len <= 1024 * kEPT) return launch_cfg<1024, true>(grid, p, stream);
-  return launch_cfg<1024, false>(grid, p, stream);
+cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream) {
+  if (p.total_q <= 0) return cudaSuccess;
+  if (max_kv_len <= 256 * 32) return launch_reg<256, 32, 2>(p, stream);
+  if (max_kv_len <= 1024 * 32) return launch_reg<1024, 32, 1>(p, stream);
+  topk_stream_kernel<1024><<<p.total_q, 1024, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa
