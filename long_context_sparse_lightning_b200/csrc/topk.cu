@@ -36,6 +36,7 @@ namespace {
 constexpr int kBins = 2048;
 constexpr int kCandCap = 512;     // boundary-bin positions ranked pairwise
 constexpr int kSegChunks = 16;    // chunks per compaction segment: 16 x 4 flags per thread
+constexpr int kMaxK = 2048;       // largest k_sel
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -78,16 +79,18 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return before + x - v;
 }
 
-template <int BLOCK>
+template <int BLOCK, int CAPW>
 struct TopkShared {
   static constexpr int NW = BLOCK / 32;
   uint32_t hist[kBins];
   float cand_v[kCandCap];
   int32_t cand_p[kCandCap];
   uint8_t cand_sel[kCandCap];
+  uint32_t selbits[CAPW > 0 ? CAPW : 1];   // verdicts of boundary-bin positions, by position
+  int32_t out_s[kMaxK];                     // the row's output, compacted before one coalesced store
   uint32_t tab[kSegChunks * NW];
+  float s_red[4][32];
   uint32_t s_warp[32];
-  float s_max[32], s_min[32];
   uint32_t s_bstar, s_above, s_cnt, s_ncand, s_total, s_digit;
   alignas(8) uint64_t bar;
 };
@@ -143,71 +146,109 @@ __device__ __forceinline__ float min_nan(float a, float b) {
 // Value-bin selection.  Returns false, having written nothing, when the row
 // holds a non-finite score or its boundary bin holds more than kCandCap
 // positions; the caller then runs select_radix.
-template <int BLOCK, int EPT, typename Get4>
-__device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, int n, int n_chunks, int k,
-                                            int32_t* __restrict__ out) {
+//
+// The histogram covers [lo, max] rather than the whole row: lo is the value a
+// normal fit of the row (mean and spread) expects about 4k positions to reach
+// (upper-tail normal quantile by the rational approximation 26.2.23 of
+// Abramowitz & Stegun).  Positions below lo cost no atomic and no ranking.  The
+// fit only has to be roughly right: when fewer than k positions reach lo, the
+// histogram is rebuilt over the full range.
+template <int BLOCK, int EPT, int CAPW, typename Get4>
+__device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& get4, int n, int n_chunks, int k,
+                                            float x0, int32_t* __restrict__ out) {
   constexpr int NW = BLOCK / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t FULL = 0xffffffffu;
   auto pos_of = [&](int v, int c) { return (v * BLOCK + tid) * 4 + c; };
 
-  // ---- range of the row (NaN-propagating, so any NaN or inf shows) ----
-  float mx = -FLT_MAX, mn = FLT_MAX;
+  // ---- range (NaN-propagating, so any NaN or inf shows); mean and spread
+  // about x0 from a sample: the first chunk and the middle one ----
+  const int v_mid = n_chunks / 2;
+  float mx = -FLT_MAX, mn = FLT_MAX, s1 = 0.f, s2 = 0.f;
   for_range<EPT>(0, n_chunks, [&](int v) {
     const float4 f = get4(v);
     const float e[4] = {f.x, f.y, f.z, f.w};
+    const bool sample = v == 0 || v == v_mid;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       if (pos_of(v, c) < n) {
         mx = max_nan(mx, e[c]);
         mn = min_nan(mn, e[c]);
+        if (sample) {
+          const float d = e[c] - x0;
+          s1 += d;
+          s2 = fmaf(d, d, s2);
+        }
       }
     }
   });
+  // butterfly reductions leave the same value in every lane (fp add commutes)
+  auto warp_all = [&](float& a, float& b, float& c, float& d) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mx = max_nan(mx, __shfl_xor_sync(FULL, mx, o));
-    mn = min_nan(mn, __shfl_xor_sync(FULL, mn, o));
-  }
+    for (int o = 16; o > 0; o >>= 1) {
+      a = max_nan(a, __shfl_xor_sync(FULL, a, o));
+      b = min_nan(b, __shfl_xor_sync(FULL, b, o));
+      c += __shfl_xor_sync(FULL, c, o);
+      d += __shfl_xor_sync(FULL, d, o);
+    }
+  };
+  warp_all(mx, mn, s1, s2);
   if (lane == 0) {
-    sh.s_max[warp] = mx;
-    sh.s_min[warp] = mn;
+    sh.s_red[0][warp] = mx;
+    sh.s_red[1][warp] = mn;
+    sh.s_red[2][warp] = s1;
+    sh.s_red[3][warp] = s2;
   }
   for (int j = tid; j < kBins; j += BLOCK) sh.hist[j] = 0u;
   if (tid == 0) sh.s_ncand = 0u;
   __syncthreads();
-  mx = sh.s_max[0];
-  mn = sh.s_min[0];
-#pragma unroll
-  for (int w = 1; w < NW; ++w) {
-    mx = max_nan(mx, sh.s_max[w]);
-    mn = min_nan(mn, sh.s_min[w]);
-  }
+  mx = lane < NW ? sh.s_red[0][lane] : -FLT_MAX;
+  mn = lane < NW ? sh.s_red[1][lane] : FLT_MAX;
+  s1 = lane < NW ? sh.s_red[2][lane] : 0.f;
+  s2 = lane < NW ? sh.s_red[3][lane] : 0.f;
+  warp_all(mx, mn, s1, s2);   // every warp reduces the same partials in the same order
   if (!(fabsf(mx) <= FLT_MAX && fabsf(mn) <= FLT_MAX)) return false;   // uniform
 
-  // Bin of a score: the integer part of 2^23 + (x - mn) * 2048 / (mx - mn),
+  float lo = mn;
+  {
+    const float f = 4.f * static_cast<float>(k) / static_cast<float>(n);
+    if (f < 0.5f) {
+      auto in_chunk = [&](int v) { return min(max(n - 4 * BLOCK * v, 0), 4 * BLOCK); };
+      const int n_sample = in_chunk(0) + (v_mid != 0 ? in_chunk(v_mid) : 0);
+      const float inv_n = 1.f / static_cast<float>(n_sample);
+      const float mean = s1 * inv_n;
+      const float var = fmaxf(s2 * inv_n - mean * mean, 0.f);
+      const float t = sqrtf(-2.f * logf(f));
+      const float z = t - (2.515517f + t * (0.802853f + t * 0.010328f)) /
+                              (1.f + t * (1.432788f + t * (0.189269f + t * 0.001308f)));
+      lo = fminf(fmaxf(mn, x0 + mean + z * sqrtf(var)), mx);
+    }
+  }
+
+  // Bin of a score x >= lo: the integer part of 2^23 + (x - lo) * 2048 / (mx - lo),
   // read from the float's bits and clamped to [0, 2047].  One rounding (fma)
   // of a function increasing in x, so the map is monotone: bins are ordered
-  // like the scores.  (The candidates inside b* are then ranked exactly, so
+  // like the scores.  (The positions inside b* are then ranked exactly, so
   // rounding only moves positions between neighbouring bins.)
-  const float scale = static_cast<float>(kBins) / (mx - mn);
-  const float off = 8388608.0f - mn * scale;
+  float scale = 0.f, off = 0.f;
   auto bin_of = [&](float x) -> int {
     const int b = static_cast<int>(__float_as_uint(__fmaf_rn(x, scale, off))) - 0x4B000000;
     return min(max(b, 0), kBins - 1);
   };
-
-  // ---- histogram ----
-  for_range<EPT>(0, n_chunks, [&](int v) {
-    const float4 f = get4(v);
-    const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll 1
+  for (int attempt = 0;; ++attempt) {
+    scale = static_cast<float>(kBins) / (mx - lo);
+    off = 8388608.0f - lo * scale;
+    // ---- histogram of the positions at or above lo ----
+    for_range<EPT>(0, n_chunks, [&](int v) {
+      const float4 f = get4(v);
+      const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      if (pos_of(v, c) < n) atomicAdd(&sh.hist[bin_of(e[c])], 1u);
-  });
-  __syncthreads();
-  // ---- bin b* with count(bins above) < k <= count(bins at or above) ----
-  {
+      for (int c = 0; c < 4; ++c)
+        if (pos_of(v, c) < n && e[c] >= lo) atomicAdd(&sh.hist[bin_of(e[c])], 1u);
+    });
+    __syncthreads();
+    // ---- bin b* with count(bins above) < k <= count(bins at or above) ----
     constexpr int BPT = kBins / BLOCK;
     uint32_t local[BPT];
     uint32_t sum = 0;
@@ -218,15 +259,22 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
     }
     uint32_t total;
     uint32_t above = block_excl_scan<BLOCK>(sum, sh.s_warp, total);
+    if (total >= static_cast<uint32_t>(k) || attempt > 0) {
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      if (above < static_cast<uint32_t>(k) && above + local[j] >= static_cast<uint32_t>(k)) {
-        sh.s_bstar = static_cast<uint32_t>(kBins - 1 - (tid * BPT + j));
-        sh.s_above = above;
-        sh.s_cnt = local[j];
+      for (int j = 0; j < BPT; ++j) {
+        if (above < static_cast<uint32_t>(k) && above + local[j] >= static_cast<uint32_t>(k)) {
+          sh.s_bstar = static_cast<uint32_t>(kBins - 1 - (tid * BPT + j));
+          sh.s_above = above;
+          sh.s_cnt = local[j];
+        }
+        above += local[j];
       }
-      above += local[j];
+      break;
     }
+    // fewer than k positions reach lo: histogram the whole row
+    lo = mn;
+    for (int j = tid; j < kBins; j += BLOCK) sh.hist[j] = 0u;
+    __syncthreads();
   }
   __syncthreads();
   const int bstar = static_cast<int>(sh.s_bstar);
@@ -241,15 +289,19 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
     for_range<EPT>(seg0, seg1, [&](int v) {
       const float4 f = get4(v);
       const float e[4] = {f.x, f.y, f.z, f.w};
+      uint32_t cs = 0, cb = 0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int pos = pos_of(v, c);
-        const int b = pos < n ? bin_of(e[c]) : -1;
-        const uint64_t bit = uint64_t(1) << (4 * (v - seg0) + c);
-        if (b > bstar) sel |= bit;
-        const bool is = b == bstar;
-        if (is) inb |= bit;
-        if (collect) {
+        const int b = (pos_of(v, c) < n && e[c] >= lo) ? bin_of(e[c]) : -1;
+        cs |= static_cast<uint32_t>(b > bstar) << c;
+        cb |= static_cast<uint32_t>(b == bstar) << c;
+      }
+      sel |= static_cast<uint64_t>(cs) << (4 * (v - seg0));
+      inb |= static_cast<uint64_t>(cb) << (4 * (v - seg0));
+      if (collect && __any_sync(FULL, cb != 0u)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool is = (cb >> c) & 1u;
           const uint32_t m = __ballot_sync(FULL, is);
           if (m != 0u) {
             const int leader = __ffs(m) - 1;
@@ -259,7 +311,7 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
             const uint32_t slot = base + __popc(m & lanemask_lt());
             if (is && slot < static_cast<uint32_t>(kCandCap)) {
               sh.cand_v[slot] = e[c];
-              sh.cand_p[slot] = pos;
+              sh.cand_p[slot] = pos_of(v, c);
             }
           }
         }
@@ -277,22 +329,29 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
       classify(seg0, min(seg0 + kSegChunks, n_chunks), true, sel, inb);
   }
   __syncthreads();
-  // rank each b* position (higher score first, then lower position); the
-  // first `rem` are selected
+  // ---- rank each b* position (higher score first, then lower position), one
+  // warp per position; the first `rem` are selected ----
   const uint32_t ncand = min(sh.s_ncand, static_cast<uint32_t>(kCandCap));
-  for (uint32_t i = tid; i < ncand; i += BLOCK) {
+  for (uint32_t i = warp; i < ncand; i += NW) {
     const float x = sh.cand_v[i];
     const int pos = sh.cand_p[i];
     uint32_t rank = 0;
-    for (uint32_t j = 0; j < ncand; ++j) {
+    for (uint32_t j = lane; j < ncand; j += 32) {
       const float y = sh.cand_v[j];
       rank += (y > x) || (y == x && sh.cand_p[j] < pos);
     }
-    sh.cand_sel[i] = rank < rem;
+    rank = __reduce_add_sync(FULL, rank);
+    if (lane == 0) {
+      if constexpr (CAPW > 0) {
+        if (rank < rem) atomicOr(&sh.selbits[pos >> 5], 1u << (pos & 31));
+      } else {
+        sh.cand_sel[i] = rank < rem;
+      }
+    }
   }
   __syncthreads();
 
-  // ---- ordered compaction, segment by segment ----
+  // ---- ordered compaction into shared memory, segment by segment ----
   uint32_t base = 0;
 #pragma unroll 1
   for (int seg0 = 0; seg0 < n_chunks; seg0 += kSegChunks) {
@@ -303,8 +362,14 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
       const int bit = __ffsll(static_cast<long long>(inb)) - 1;
       inb &= inb - 1;
       const int pos = ((seg0 + (bit >> 2)) * BLOCK + tid) * 4 + (bit & 3);
-      for (uint32_t j = 0; j < ncand; ++j)
-        if (sh.cand_p[j] == pos && sh.cand_sel[j]) sel |= uint64_t(1) << bit;
+      bool chosen = false;
+      if constexpr (CAPW > 0) {
+        chosen = (sh.selbits[pos >> 5] >> (pos & 31)) & 1u;
+      } else {
+        for (uint32_t j = 0; j < ncand; ++j)
+          if (sh.cand_p[j] == pos) chosen = sh.cand_sel[j];
+      }
+      if (chosen) sel |= uint64_t(1) << bit;
     }
     for_range<EPT>(seg0, seg1, [&](int v) {
       const uint32_t fl = static_cast<uint32_t>(sel >> (4 * (v - seg0))) & 15u;
@@ -349,13 +414,17 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         if ((fl >> c) & 1u) {
-          if (o < static_cast<uint32_t>(k)) out[o] = pos_of(v, c);
+          if (o < static_cast<uint32_t>(k)) sh.out_s[o] = pos_of(v, c);
           ++o;
         }
       }
     });
     base = sh.s_total;
     __syncthreads();
+  }
+  for (int j = tid; j < k; j += BLOCK) out[j] = sh.out_s[j];
+  if constexpr (CAPW > 0) {
+    for (uint32_t i = tid; i < ncand; i += BLOCK) sh.selbits[sh.cand_p[i] >> 5] = 0u;
   }
   return true;
 }
@@ -364,8 +433,8 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK>& sh, Get4&& get4, 
 // warp-aggregated histogram updates), for rows select_fast declines: finds the
 // threshold key T and how many T-valued positions are needed, then writes the
 // selected positions in ascending order.
-template <int BLOCK, typename Get4>
-__device__ __noinline__ void select_radix(TopkShared<BLOCK>& sh, Get4 get4, int n, int n_chunks, int k,
+template <int BLOCK, int CAPW, typename Get4>
+__device__ __noinline__ void select_radix(TopkShared<BLOCK, CAPW>& sh, Get4 get4, int n, int n_chunks, int k,
                                           int32_t* __restrict__ out) {
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t FULL = 0xffffffffu;
@@ -498,7 +567,7 @@ __device__ __forceinline__ void issue_row_copy(float* buf, const float* row, int
 
 template <int BLOCK, int EPT>
 constexpr size_t reg_smem_bytes() {
-  return ((sizeof(TopkShared<BLOCK>) + 127) / 128) * 128 + static_cast<size_t>(BLOCK) * EPT * sizeof(float);
+  return ((sizeof(TopkShared<BLOCK, BLOCK * EPT / 32>) + 127) / 128) * 128 + static_cast<size_t>(BLOCK) * EPT * sizeof(float);
 }
 
 // Persistent kernel for rows of up to BLOCK*EPT positions: the row being
@@ -507,9 +576,10 @@ constexpr size_t reg_smem_bytes() {
 template <int BLOCK, int EPT, int MIN_CTAS>
 __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkParams p) {
   extern __shared__ __align__(128) uint8_t dyn[];
-  auto& sh = *reinterpret_cast<TopkShared<BLOCK>*>(dyn);
-  float* buf = reinterpret_cast<float*>(dyn + ((sizeof(TopkShared<BLOCK>) + 127) / 128) * 128);
   constexpr int CAP = BLOCK * EPT;
+  using Shared = TopkShared<BLOCK, CAP / 32>;
+  auto& sh = *reinterpret_cast<Shared*>(dyn);
+  float* buf = reinterpret_cast<float*>(dyn + ((sizeof(Shared) + 127) / 128) * 128);
   const int k = p.k_sel;
   const int tid = threadIdx.x;
   const int G = gridDim.x;
@@ -519,6 +589,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
     mbar_init(&sh.bar, 1);
     fence_mbar_init();
   }
+  for (int j = tid; j < CAP / 32; j += BLOCK) sh.selbits[j] = 0u;
   __syncthreads();
 
   auto needs_copy = [&](int r, int& n) { return r < p.total_q && row_info(p, r, n) && n > k && n <= CAP; };
@@ -566,6 +637,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
       x[4 * v + 2] = f.z;
       x[4 * v + 3] = f.w;
     }
+    const float x0 = buf[0];
     __syncthreads();   // the buffer is free: start the next row's copy
     {
       int nn;
@@ -575,7 +647,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
       }
     }
     auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
-    if (!select_fast<BLOCK, EPT>(sh, get4, n, n_chunks, k, out)) {
+    if (!select_fast<BLOCK, EPT>(sh, get4, n, n_chunks, k, x0, out)) {
       const GlobalRow<BLOCK> g{reinterpret_cast<const float4*>(scores + static_cast<int64_t>(r) * p.ld), n_vec};
       select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
     }
@@ -585,7 +657,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
 // One CTA per row for rows longer than the register path holds.
 template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) {
-  __shared__ TopkShared<BLOCK> sh;
+  __shared__ TopkShared<BLOCK, 0> sh;
   const int k = p.k_sel;
   const int r = blockIdx.x;
   if (error_pending(p.err)) return;
@@ -603,7 +675,8 @@ __global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) 
   const int n_vec = (n + 3) >> 2;
   const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
   const GlobalRow<BLOCK> g{row4, n_vec};
-  if (!select_fast<BLOCK, 0>(sh, g, n, n_chunks, k, out)) select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
+  if (!select_fast<BLOCK, 0>(sh, g, n, n_chunks, k, __ldg(p.scores + static_cast<int64_t>(r) * p.ld), out))
+    select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
 }
 
 int sm_count() {
