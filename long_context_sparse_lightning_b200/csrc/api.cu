@@ -200,19 +200,16 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   const int64_t gx = int64_t(2) * b->max_q_per_seq * sp.nsplit;
   if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
+  dsa::MlaMaps maps;
+  if (!dsa::make_mla_maps(&maps, q, out, b->total_q, n_heads)) return DSA_ERR_CUDA;
   if (mla_copy(b, k_sel)) {
     uint16_t* kv16 = reinterpret_cast<uint16_t*>(part + mla_part_bytes(b, k_sel));
     const int64_t n = b->total_keys * 576;
     if (dsa::launch_latent_to_fp16(static_cast<const uint16_t*>(kv), kv16, n, stream) != cudaSuccess)
       return DSA_ERR_CUDA;
-    CUtensorMap ml, mr;
-    if (!make_tmap_2d(&ml, kv16, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(b->total_keys), 576, 1, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&mr, kv16, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(b->total_keys), 576, 1, 32,
-                      CU_TENSOR_MAP_SWIZZLE_64B))
-      return DSA_ERR_CUDA;
-    if (dsa::launch_sparse_mla_tma(grid, p, ml, mr, stream) != cudaSuccess) return DSA_ERR_CUDA;
-  } else if (dsa::launch_sparse_mla(grid, p, stream) != cudaSuccess) {
+    p.kv = kv16;
+    if (dsa::launch_sparse_mla_fp16(grid, p, maps, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  } else if (dsa::launch_sparse_mla(grid, p, maps, stream) != cudaSuccess) {
     return DSA_ERR_CUDA;
   }
   if (sp.nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
@@ -238,6 +235,16 @@ dsa_status_t check_mla_args(const void* q, int n_heads, const void* kv, int k_se
 }
 
 }  // namespace
+
+namespace dsa {
+bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads) {
+  const uint64_t rows = static_cast<uint64_t>(total_q) * static_cast<uint64_t>(n_heads);
+  const uint32_t h = static_cast<uint32_t>(n_heads);
+  return make_tmap_2d(&m->q_lat, q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 576, h, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tmap_2d(&m->q_rope, q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 576, h, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_tmap_2d(&m->out, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 512, h, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+}  // namespace dsa
 
 extern "C" {
 

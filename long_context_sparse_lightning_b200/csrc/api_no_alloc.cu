@@ -112,7 +112,9 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   const int64_t gx = int64_t(2) * b->max_q_per_seq * nsplit;
   if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
-  if (dsa::launch_sparse_mla(grid, p, st) != cudaSuccess) return DSA_ERR_CUDA;
+  dsa::MlaMaps maps;
+  if (!dsa::make_mla_maps(&maps, q, out, b->total_q, n_heads)) return DSA_ERR_CUDA;
+  if (dsa::launch_sparse_mla(grid, p, maps, st) != cudaSuccess) return DSA_ERR_CUDA;
   if (nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }

@@ -54,7 +54,7 @@ struct MlaParams {
   const int32_t* kv_len = nullptr;
   const int64_t* kv_start = nullptr;
   const uint16_t* q = nullptr;        // bf16 [total_q, H, 576]
-  const uint16_t* kv = nullptr;       // bf16 [total_keys, 576]
+  const uint16_t* kv = nullptr;       // [total_keys, 576]: bf16 cache, or its fp16 copy
   const int32_t* idx = nullptr;       // [total_q, k_sel]
   int64_t total_keys = 0;
   int32_t k_sel = 0;
@@ -76,14 +76,24 @@ int mla_keys_per_split(int k_sel, int nsplit);
 // selections reuse each latent row often enough to amortise the copy.
 bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_sel);
 size_t mla_smem_bytes();
-// Selected rows gathered with 16-byte loads and converted to fp16 on the way
-// into shared memory (no extra buffers).
-cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, cudaStream_t stream);
-// Selected rows gathered by TMA from `kv16`, an fp16 copy of the latent cache
-// described by the two tensor maps (64-column / 128-byte-swizzled boxes for the
-// latent dims, 32-column / 64-byte-swizzled boxes for the RoPE dims).
-cudaError_t launch_sparse_mla_tma(dim3 grid, const MlaParams& p, const CUtensorMap& map_lat,
-                                  const CUtensorMap& map_rope, cudaStream_t stream);
+// TMA descriptors of the sparse MLA kernel (bf16 bits as 16-bit elements):
+//   q_lat  over q viewed as [total_q * H, 576], box [H rows x 64 cols], 128-byte swizzle
+//   q_rope the same tensor, box [H rows x 32 cols], 64-byte swizzle
+//   out    over out viewed as [total_q * H, 512], box [H rows x 64 cols], 128-byte swizzle
+struct MlaMaps {
+  CUtensorMap q_lat;
+  CUtensorMap q_rope;
+  CUtensorMap out;
+};
+// Encodes the three descriptors for q [total_q * n_heads, 576] and out
+// [total_q * n_heads, 512]; false if the driver refuses them.
+bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads);
+// p.kv is the bf16 cache: selected rows are gathered with 16-byte loads and
+// converted to fp16 in shared memory (no extra buffers).
+cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
+// p.kv is an fp16 copy of the cache (launch_latent_to_fp16): rows are
+// gathered ready for the MMAs.
+cudaError_t launch_sparse_mla_fp16(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
 cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream);
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream);
 

@@ -20,10 +20,13 @@
 // K-major for Q.C^T, MN-major for P.V).
 //
 // Per tile of 64 selected entries:
-//   gather     fp16 copy of the latent cache + TMA gather4 (prefill: rows are
-//              reused across many tokens), or 6 producer warps copying bf16 rows
-//              with 16-byte cp.async into place and converting them to fp16 in
-//              shared memory (decode); 4-stage ring;
+//   gather     7 producer warps copy each row's 16-byte units with cp.async
+//              straight into their swizzled slots, from an fp16 copy of the
+//              latent cache (prefill: rows are reused across many tokens) or
+//              from the bf16 cache with an in-place conversion to fp16
+//              (decode); 4-stage ring.  (TMA gather4 moves 4 rows x 128 B per
+//              instruction and measured ~6 B/clk per SM on this pattern;
+//              16-byte cp.async from 7 warps sustains several times that.)
 //   MMA warp   S_r = Q_r . C_r^T (M=128, N=64, K=288) then O_r += P . V_r (N=256);
 //   softmax    8 warps, two per TMEM lane quarter, each half owning 32 of the 64
 //              columns: each warp ships its 2 KB of partial scores (fp16; both
@@ -42,8 +45,6 @@
 // normalised partial output and its log-sum-exp, merged by mla_combine_kernel.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-
-#include <cstring>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -76,8 +77,10 @@ constexpr int kSmem = OFF_MISC + 64 + 1024;
 
 constexpr int kUnitsPerRow = 36;                     // 16-byte units of a row's 288-dim half
 constexpr int kTileUnits = kTileKeys * kUnitsPerRow; // 2304
+constexpr int kQBox = 16384;                         // one 128-row x 128-byte TMA box of Q or O
 
 struct Bars {
+  uint64_t q_tma;           // this CTA's Q slice landed in shared memory (TMA)
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
@@ -88,14 +91,18 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "");
 
-template <bool TMA>
+// Warp roles: 7 producer warps, 1 MMA warp, 8 softmax warps (two warpgroups,
+// so warp w reaches TMEM lane quarter w % 4 as the hardware requires).
 struct Cfg {
-  static constexpr int NPROD = TMA ? 1 : 6;          // producer warps
+  static constexpr int NPROD = 7;
   static constexpr int MMA_WARP = NPROD;
-  static constexpr int SOFT0 = NPROD + 1;            // 8 softmax warps follow
+  static constexpr int SOFT0 = NPROD + 1;
   static constexpr int THREADS = (NPROD + 1 + 8) * 32;
-  static constexpr int UNITS = TMA ? 1 : kTileUnits / (NPROD * 32);   // 12 per producer thread
+  static constexpr int PTHREADS = NPROD * 32;
 };
+static_assert(Cfg::SOFT0 % 4 == 0, "softmax warps must start a warpgroup");
+static_assert(2048 % Cfg::THREADS == 0, "index staging assumes whole warps per pass");
+static_assert(4 * kQBox + 128 * 64 <= 2 * KV_STAGE, "Q slice must fit ring stages 2-3");
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   const float lo = __uint_as_float(w << 16);
@@ -127,7 +134,7 @@ __device__ __forceinline__ int unit_dim(int u, uint32_t r) {
 
 // Shared-memory offset of unit u of row j inside a stage: units 0..31 form four
 // 64-dim chunks (8 KB each, 128-byte swizzle), units 32..35 the RoPE chunk
-// (64-byte swizzle) -- the layouts TMA writes for 128/64-byte boxes.
+// (64-byte swizzle): the canonical K-major SW128 / SW64 operand layouts.
 __device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
   if (u < 32) {
     const int c = u >> 3, cu = u & 7;
@@ -137,11 +144,12 @@ __device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
   return KV_ROPE + j * 64 + ((ru ^ ((j >> 1) & 3)) << 4);
 }
 
-template <bool TMA>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1)
-    sparse_mla_kernel(const MlaParams p, const __grid_constant__ CUtensorMap map_lat,
-                      const __grid_constant__ CUtensorMap map_rope) {
-  using C = Cfg<TMA>;
+// FP16_SRC: p.kv is an fp16 copy of the latent cache (rows land ready for the
+// MMAs); otherwise p.kv is the bf16 cache and producers convert in place.
+template <bool FP16_SRC>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
+    sparse_mla_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
+  using C = Cfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -181,28 +189,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
   const uint32_t lane = lane_id();
   const int tid = threadIdx.x;
 
-  // ---- this split's selected positions (invalid -> -1) and per-32 validity bits ----
-  if (tid == 0) *s_last = -1;
-  __syncthreads();
-  const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
-  int my_last = -1;
-  for (int j = tid; j < 2048; j += C::THREADS) {
-    int v = -1;
-    if (j < e_count) {
-      v = __ldg(&idx_row[j]);
-      if (v < 0 || v >= kv) v = -1;
-    }
-    sIdx[j] = v;
-    const uint32_t bits = __ballot_sync(0xffffffffu, v >= 0);
-    if (lane == 0) sValid[j >> 5] = bits;
-    if (v >= 0) my_last = j;
-  }
-  if (my_last >= 0) atomicMax(s_last, my_last);
-
+  // ---- barriers, then this CTA's Q slice by TMA into ring stages 2-3 (free
+  // until the producers' third tile, which waits for q_full) ----
+  uint8_t* sQ = sKV + 2 * KV_STAGE;
   if (tid == 0) {
+    *s_last = -1;
+    mbar_init(&bar->q_tma, 1);
     mbar_init(&bar->q_full, 8);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar->kv_full[s], TMA ? 1 : C::NPROD);
+      mbar_init(&bar->kv_full[s], C::NPROD);
       mbar_init(&bar->kv_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
@@ -215,7 +210,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->red, 256);
     fence_mbar_init();
+    mbar_arrive_expect_tx(&bar->q_tma, static_cast<uint32_t>(H) * (4 * 128 + 64));
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      tma_load_2d(sQ + c * kQBox, &maps.q_lat, &bar->q_tma, static_cast<int>(rank) * 256 + c * 64, row * H);
+    tma_load_2d(sQ + 4 * kQBox, &maps.q_rope, &bar->q_tma, 512 + static_cast<int>(rank) * 32, row * H);
   }
+  __syncthreads();
+
+  // ---- this split's selected positions (invalid -> -1) and per-32 validity bits ----
+  const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
+  int my_last = -1;
+  {
+    constexpr int PER = (2048 + C::THREADS - 1) / C::THREADS;
+    int v[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {      // all loads first: one memory latency
+      const int j = tid + q * C::THREADS;
+      v[q] = (j < 2048 && j < e_count) ? __ldg(&idx_row[j]) : -1;
+    }
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int j = tid + q * C::THREADS;
+      if (j < 2048) {
+        const int e = (v[q] < 0 || v[q] >= kv) ? -1 : v[q];
+        sIdx[j] = e;
+        const uint32_t bits = __ballot_sync(0xffffffffu, e >= 0);
+        if (lane == 0) sValid[j >> 5] = bits;
+        if (e >= 0) my_last = j;
+      }
+    }
+  }
+  if (my_last >= 0) atomicMax(s_last, my_last);
+
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -229,89 +256,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
 
   if (warp < C::NPROD) {
     // ------------------------------------------------------------ producers --
-    if constexpr (TMA) {
-      if (n_tiles > 0 && elect_one()) {
-        prefetch_tmap(&map_lat);
-        prefetch_tmap(&map_rope);
-        for (int i = 0; i < n_tiles; ++i) {
-          const int st = i % kStages;
-          if (!mbar_wait(&bar->kv_empty[st], ((i / kStages) & 1) ^ 1, p.budget)) {
-            report_error(p.err, kDevErrTimeout, 310, i);
-            break;
-          }
-          mbar_arrive_expect_tx(&bar->kv_full[st], KV_STAGE);
-          uint8_t* base = sKV + st * KV_STAGE;
-          const int* e = sIdx + i * kTileKeys;
-#pragma unroll 1
-          for (int g4 = 0; g4 < 16; ++g4) {
-            const int y0 = static_cast<int>(kstart + max(e[4 * g4 + 0], 0));
-            const int y1 = static_cast<int>(kstart + max(e[4 * g4 + 1], 0));
-            const int y2 = static_cast<int>(kstart + max(e[4 * g4 + 2], 0));
-            const int y3 = static_cast<int>(kstart + max(e[4 * g4 + 3], 0));
+    // Each 16-byte unit goes straight to its swizzled slot with cp.async;
+    // consecutive lanes take consecutive units of a row, so one warp request
+    // covers a few whole 128-byte lines.  bf16 sources are converted to fp16 in
+    // place by the thread that loaded them.  Two tiles ahead.
+    if (n_tiles > 0) {
+      const uint8_t* kvbase = reinterpret_cast<const uint8_t*>(p.kv + kstart * 576);
+      // this thread's units (the same slots in every tile): unit g = tid + m * PTHREADS
+      // of the tile is row j = g / 36, 16-byte unit u = g % 36
+      constexpr int UPT = (kTileUnits + C::PTHREADS - 1) / C::PTHREADS;
+      uint32_t soff[UPT], goff[UPT], jrow[UPT];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              tma_gather4(base + c * 8192 + g4 * 512, &map_lat, &bar->kv_full[st],
-                          static_cast<int>(rank) * 256 + c * 64, y0, y1, y2, y3);
+      for (int m = 0; m < UPT; ++m) {
+        const int g = min(tid + m * C::PTHREADS, kTileUnits - 1);
+        const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
+        soff[m] = tile_unit_offset(j, u);
+        goff[m] = static_cast<uint32_t>(unit_dim(u, rank)) * 2u;
+        jrow[m] = static_cast<uint32_t>(j);
+      }
+      auto mine = [&](int m) { return m + 1 < UPT || tid + m * C::PTHREADS < kTileUnits; };
+      bool ok = true;
+      auto issue = [&](int tile) {
+        const int st = tile % kStages;
+        if (ok && !mbar_wait(&bar->kv_empty[st], ((tile / kStages) & 1) ^ 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 311, tile);
+          ok = false;
+        }
+        // stages 2-3 hold the Q slice until the softmax warps have moved it to TMEM
+        if (ok && (tile == 2 || tile == 3) && !mbar_wait(&bar->q_full, 0, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 312, tile);
+          ok = false;
+        }
+        if (ok) {
+          const uint32_t base = smem_u32(sKV + st * KV_STAGE);
+          const int32_t* e = sIdx + tile * kTileKeys;
+#pragma unroll
+          for (int m = 0; m < UPT; ++m) {
+            if (mine(m)) {
+              const int pos = max(e[jrow[m]], 0);
+              cp_async_16(base + soff[m], kvbase + static_cast<int64_t>(pos) * 1152 + goff[m]);
             }
-            tma_gather4(base + KV_ROPE + g4 * 256, &map_rope, &bar->kv_full[st], 512 + static_cast<int>(rank) * 32,
-                        y0, y1, y2, y3);
           }
         }
-      }
-    } else {
-      if (n_tiles > 0) {
-        // cp.async each 16-byte unit straight to its swizzled slot (bf16), then
-        // convert the thread's own units to fp16 in place; two tiles ahead.
-        const uint16_t* kvbase = p.kv + kstart * 576;
-        bool ok = true;
-        auto issue = [&](int tile) {
-          const int st = tile % kStages;
-          if (ok && !mbar_wait(&bar->kv_empty[st], ((tile / kStages) & 1) ^ 1, p.budget)) {
-            report_error(p.err, kDevErrTimeout, 311, tile);
-            ok = false;
-          }
-          if (ok) {
-            const uint32_t base = smem_u32(sKV + st * KV_STAGE);
-#pragma unroll
-            for (int m = 0; m < C::UNITS; ++m) {
-              const int g = tid + m * C::NPROD * 32;
-              const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
-              const int s = sIdx[tile * kTileKeys + j];
-              const int pos = s >= 0 ? s : 0;
-              cp_async_16(base + tile_unit_offset(j, u), kvbase + static_cast<int64_t>(pos) * 576 + unit_dim(u, rank));
-            }
-          }
-          cp_async_commit();
-        };
-        auto convert = [&](int tile) {
+        cp_async_commit();
+      };
+      auto land = [&](int tile) {
+        if constexpr (!FP16_SRC) {
           uint8_t* base = sKV + (tile % kStages) * KV_STAGE;
 #pragma unroll
-          for (int m = 0; m < C::UNITS; ++m) {
-            const int g = tid + m * C::NPROD * 32;
-            uint4* q = reinterpret_cast<uint4*>(base + tile_unit_offset(g / kUnitsPerRow, g % kUnitsPerRow));
-            *q = cvt_unit(*q);
+          for (int m = 0; m < UPT; ++m) {
+            if (mine(m)) {
+              uint4* q = reinterpret_cast<uint4*>(base + soff[m]);
+              *q = cvt_unit(*q);
+            }
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar->kv_full[tile % kStages]);
-        };
-        // convert tile i before waiting for tile i+2's ring slot: that slot is
-        // freed by P.V of tile i-2, which runs after Q.C^T of tile i, which
-        // needs tile i converted
-        issue(0);
-        if (n_tiles > 1) issue(1);
-        for (int i = 0; i < n_tiles; ++i) {
-          if (i + 1 < n_tiles) {
-            cp_async_wait<1>();
-          } else {
-            cp_async_wait<0>();
-          }
-          if (!ok) break;
-          convert(i);
-          if (i + 2 < n_tiles) issue(i + 2);
         }
-        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->kv_full[tile % kStages]);
+      };
+      // land tile i before waiting for tile i+2's ring slot: that slot is
+      // freed by P.V of tile i-2, which runs after Q.C^T of tile i, which
+      // needs tile i landed
+      issue(0);
+      if (n_tiles > 1) issue(1);
+      for (int i = 0; i < n_tiles; ++i) {
+        if (i + 1 < n_tiles) {
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+        if (!ok) break;
+        land(i);
+        if (i + 2 < n_tiles) issue(i + 2);
       }
+      cp_async_wait<0>();
     }
   } else if (warp == C::MMA_WARP) {
     // ----------------------------------------------------------- MMA issuer --
@@ -442,14 +461,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
       return true;
     };
 
+    // every softmax warp waits for the Q slice, also when there is nothing to
+    // attend, so no TMA write is still in flight when the CTA exits
+    if (!wwait(&bar->q_tma, 0, false, 338, 0)) ok = false;
     if (n_tiles > 0) {
       // Q_r row h into TMEM: this half writes dims [144g, 144g+144) = columns [72g, 72g+72)
       uint32_t qv[72];
-      const uint16_t* qrow = p.q + (static_cast<int64_t>(row) * H + h) * 576;
 #pragma unroll
       for (int m = 0; m < 18; ++m) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (h < H) v = cvt_unit(__ldg(reinterpret_cast<const uint4*>(qrow + unit_dim(18 * g + m, rank))));
+        const int u = 18 * g + m;        // unit of the CTA's 288 dims: 0..31 latent, 32..35 RoPE
+        const uint32_t off = u < 32 ? (u >> 3) * kQBox + h * 128 + (((u & 7) ^ (h & 7)) << 4)
+                                    : 4 * kQBox + h * 64 + (((u - 32) ^ ((h >> 1) & 3)) << 4);
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (ok && h < H) raw = *reinterpret_cast<const uint4*>(sQ + off);
+        const uint4 v = cvt_unit(raw);
         qv[4 * m + 0] = v.x;
         qv[4 * m + 1] = v.y;
         qv[4 * m + 2] = v.z;
@@ -586,7 +611,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
     const float inv_l = any ? 1.f / l : 0.f;
     const float lse_val = any ? (m_run + __log2f(l)) * 0.69314718055994531f : NEG_INF;
     if (p.nsplit == 1) {
-      uint16_t* orow = p.out + (static_cast<int64_t>(row) * H + h) * 512 + rank * 256 + 128 * g;
+      // O / l as bf16 into ring stages 0-1 (idle now) in the 128-byte-swizzled
+      // layout of four [H x 64-dim] TMA boxes, then one thread stores the boxes:
+      // whole rows leave the SM instead of 16-byte pieces strided by a head row.
+      uint8_t* sO = sKV;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
@@ -598,6 +626,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
           for (int j = 0; j < 32; ++j) o[j] = 0u;
         }
         if (h < H) {
+          const int bx = 2 * g + (c >> 1), ub = (c & 1) * 4;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t w4[4];
@@ -607,9 +636,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<TMA>::THREADS, 1
                                                              __uint_as_float(o[8 * q + 2 * e + 1]) * inv_l);
               w4[e] = *reinterpret_cast<const uint32_t*>(&v);
             }
-            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<uint4*>(sO + bx * kQBox + h * 128 + (((ub + q) ^ (h & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar->red);
+      const bool staged = wwait(&bar->red, (n_tiles + 1) & 1, false, 339, n_tiles);
+      if (staged && sw == 0 && lane == 0) {
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx)
+          tma_store_2d(&maps.out, sO + bx * kQBox, static_cast<int>(rank) * 256 + bx * 64, row * H);
+        bulk_commit_group();
+        bulk_wait_all();
       }
       if (rank == 0 && g == 0 && h < H && p.lse != nullptr) p.lse[static_cast<int64_t>(row) * H + h] = lse_val;
     } else {
@@ -691,13 +731,12 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   }
 }
 
-template <bool TMA>
-cudaError_t launch_variant(dim3 grid, const MlaParams& p, const CUtensorMap& ml, const CUtensorMap& mr,
-                           cudaStream_t stream) {
+template <bool FP16_SRC>
+cudaError_t launch_variant(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
   cudaError_t e =
-      cudaFuncSetAttribute(sparse_mla_kernel<TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+      cudaFuncSetAttribute(sparse_mla_kernel<FP16_SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  sparse_mla_kernel<TMA><<<grid, Cfg<TMA>::THREADS, kSmem, stream>>>(p, ml, mr);
+  sparse_mla_kernel<FP16_SRC><<<grid, Cfg::THREADS, kSmem, stream>>>(p, maps);
   return cudaGetLastError();
 }
 
@@ -727,15 +766,12 @@ bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_se
 
 size_t mla_smem_bytes() { return kSmem; }
 
-cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, cudaStream_t stream) {
-  CUtensorMap unused;
-  std::memset(&unused, 0, sizeof(unused));
-  return launch_variant<false>(grid, p, unused, unused, stream);
+cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+  return launch_variant<false>(grid, p, maps, stream);
 }
 
-cudaError_t launch_sparse_mla_tma(dim3 grid, const MlaParams& p, const CUtensorMap& map_lat,
-                                  const CUtensorMap& map_rope, cudaStream_t stream) {
-  return launch_variant<true>(grid, p, map_lat, map_rope, stream);
+cudaError_t launch_sparse_mla_fp16(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+  return launch_variant<true>(grid, p, maps, stream);
 }
 
 cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream) {
