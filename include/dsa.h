@@ -117,8 +117,9 @@ DSA_API dsa_status_t dsa_indexer_scores(const dsa_batch_t* batch, const void* q_
 
 /* Top-k positions per query row.
  *   scores [total_q, ld_scores] fp32 (only s <= t is read)
- *   idx    [total_q, k_sel] int32 out: the selected positions (ties: lower s
- *          first), then -1 padding when t + 1 < k_sel.
+ *   idx    [total_q, k_sel] int32 out: the k_sel highest-scoring positions
+ *          (equal scores: the lower s wins; -0 and +0 are equal) in ascending
+ *          order of s, then -1 padding when t + 1 < k_sel.
  *   1 <= k_sel <= 2048. */
 DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int64_t ld_scores, int32_t k_sel,
                       int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);

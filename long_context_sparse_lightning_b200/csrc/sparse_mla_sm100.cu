@@ -41,6 +41,11 @@
 // noise costs ~1e-3 mean relative error on the bf16 output; fp16 keeps ~1e-4.
 // The conversion of q and the latent entries is exact in the normal fp16 range.
 //
+// Per token, around the tile loop: the CTA's Q slice arrives by TMA boxes into
+// ring stages 2-3 (converted to fp16 into TMEM by the softmax warps before the
+// producers reuse those stages), and the bf16 output leaves by TMA box stores
+// staged, swizzled, in the idle ring.
+//
 // Decode shapes split a token's selection over several pairs; each writes a
 // normalised partial output and its log-sum-exp, merged by mla_combine_kernel.
 #include <cuda_bf16.h>
