@@ -61,7 +61,7 @@ constexpr int kTileKeys = 64;
 constexpr int kStages = 4;
 constexpr int KV_STAGE = 36864;          // 64 rows x (4 x 128 B latent + 64 B RoPE)
 constexpr int KV_ROPE = 32768;
-constexpr int XBLK = 2048;               // one softmax warp's partial scores: 32 heads x 32 keys fp16
+constexpr int XBLK = 2048;               // one softmax warp's partial scores: 16 heads x 64 keys fp16
 constexpr int XBUF = 8 * XBLK;           // one tile's partial scores of all 8 softmax warps
 
 constexpr uint32_t TM_O = 0;
@@ -75,9 +75,8 @@ constexpr int OFF_STG = kStages * KV_STAGE;          // 147456: outgoing partial
 constexpr int OFF_X = OFF_STG + 2 * XBUF;            // 180224: incoming partial scores, 2 buffers
 constexpr int OFF_IDX = OFF_X + 2 * XBUF;            // 212992: int32[2048]
 constexpr int OFF_VALID = OFF_IDX + 2048 * 4;        // 221184: uint32[64] validity bits
-constexpr int OFF_RED = OFF_VALID + 64 * 4;          // 221440: float[2][2][128] row maxima, float[2][128] sums
-constexpr int OFF_BAR = OFF_RED + 6 * 128 * 4;       // 224512
-constexpr int OFF_MISC = OFF_BAR + 256;
+constexpr int OFF_BAR = OFF_VALID + 64 * 4;          // 221440
+constexpr int OFF_MISC = OFF_BAR + 512;
 constexpr int kSmem = OFF_MISC + 64 + 1024;
 
 constexpr int kUnitsPerRow = 36;                     // 16-byte units of a row's 288-dim half
@@ -90,11 +89,11 @@ struct Bars {
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full, s_empty;
-  uint64_t x_full[2], x_free[2];
+  uint64_t x_full[2][8], x_free[2][8];   // per buffer and softmax warp
   uint64_t p_full, pv_done;
-  uint64_t red;            // the two column halves' row maxima / sums are in shared memory
+  uint64_t red;            // all softmax warps have staged the output
 };
-static_assert(sizeof(Bars) <= 256, "");
+static_assert(sizeof(Bars) <= 512, "");
 
 // Warp roles: 7 producer warps, 1 MMA warp, 8 softmax warps (two warpgroups,
 // so warp w reaches TMEM lane quarter w % 4 as the hardware requires).
@@ -185,7 +184,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   uint8_t* sKV = sm + OFF_KV;
   int32_t* sIdx = reinterpret_cast<int32_t*>(sm + OFF_IDX);
   uint32_t* sValid = reinterpret_cast<uint32_t*>(sm + OFF_VALID);
-  float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
   Bars* bar = reinterpret_cast<Bars*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   int32_t* s_last = reinterpret_cast<int32_t*>(sm + OFF_MISC + 4);
@@ -208,8 +206,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_empty, 8);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->x_full[i], 8);    // one expect_tx arrival per receiving warp + 16 KB of bulk copies
-      mbar_init(&bar->x_free[i], 8);    // one remote arrival per peer warp once it has read the buffer
+      for (int w = 0; w < 8; ++w) {
+        mbar_init(&bar->x_full[i][w], 1);   // the receiving warp's expect_tx arrival + the peer's 2 KB copy
+        mbar_init(&bar->x_free[i][w], 1);   // the peer warp's remote arrival once it has read the block
+      }
     }
     mbar_init(&bar->p_full, 8);
     mbar_init(&bar->pv_done, 1);
@@ -393,29 +393,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- softmax --
+    // Warp sw owns 16 heads -- TMEM lanes [32q + 16*(sw/4), +16) of its lane
+    // quarter q = warp % 4 -- across all 64 columns of a tile, read with the
+    // .16x256b shape: lane t holds heads rA = L + t/4 and rB = rA + 8, keys
+    // 8k + 2(t%4) + {0, 1} for k = 0..7.  A head's 64 scores sit in the 4 lanes
+    // of one group, so row max and sum need two shuffles and no other warp.
     const int sw = static_cast<int>(warp) - C::SOFT0;   // 0..7
-    const int g = sw >> 2;                               // column half: keys [32g, 32g+32) of a tile
     const uint32_t quarter = warp & 3u;
-    const int h = static_cast<int>(quarter * 32 + lane);
-    const uint32_t lane_base = tmem + ((quarter * 32u) << 16);
-    // partial-score blocks: this warp owns 2 KB (32 heads x 32 keys, fp16) per
-    // tile; the peer's warp with the same (g, quarter) fills the same block of
-    // our receive buffer.  16-byte unit q of lane l sits at unit q ^ ((l>>1)&3).
-    const int blk = g * 4 + static_cast<int>(quarter);
-    uint32_t uoff[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) uoff[q] = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
-    const uint32_t stg_base = smem_u32(sm + OFF_STG) + blk * XBLK;
-    const uint32_t x_base = smem_u32(sm + OFF_X) + blk * XBLK;
+    const int L = static_cast<int>(quarter) * 32 + 16 * (sw >> 2);
+    const int hA = L + static_cast<int>(lane >> 2), hB = hA + 8;
+    const int ku = 2 * static_cast<int>(lane & 3u);     // this lane's key offset inside each group of 8
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(L) << 16);
+    // partial-score blocks: 2 KB per warp per tile; lane l's 16-byte unit k at k*512 + l*16
+    const uint32_t stg_base = smem_u32(sm + OFF_STG) + sw * XBLK;
+    const uint32_t x_base = smem_u32(sm + OFF_X) + sw * XBLK;
     const uint32_t x_base_remote = mapa_shared(x_base, peer);
-    const uint32_t x_full_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0]), peer),
-                                       mapa_shared(smem_u32(&bar->x_full[1]), peer)};
-    const uint32_t x_free_remote[2] = {mapa_shared(smem_u32(&bar->x_free[0]), peer),
-                                       mapa_shared(smem_u32(&bar->x_free[1]), peer)};
+    const uint32_t x_full_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0][sw]), peer),
+                                       mapa_shared(smem_u32(&bar->x_full[1][sw]), peer)};
+    const uint32_t x_free_remote[2] = {mapa_shared(smem_u32(&bar->x_free[0][sw]), peer),
+                                       mapa_shared(smem_u32(&bar->x_free[1][sw]), peer)};
     const float NEG_INF = __int_as_float(0xff800000);
     const float scale = p.scale_log2;
-    float m_run = NEG_INF;     // running max (log2 domain), refreshed lazily; identical in both halves
-    float l_run = 0.f;         // partial row sum over this half's columns
+    float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
+    float l_runA = 0.f, l_runB = 0.f;           // this lane's share of the row sums
     bool ok = true;
     // bounded wait polled by lane 0; every lane gets the same outcome and is
     // ordered after lane 0's acquire by the warp barrier
@@ -429,13 +429,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       __syncwarp();
       return r != 0;
     };
-    // S(t) of head h, columns [32g, 32g+32), rounded to fp16 pairs (the peer
-    // receives exactly these values, so both CTAs add the same two numbers)
+    // S(t) of this warp's 16 heads, rounded to fp16 pairs (the peer receives
+    // exactly these values, so both CTAs add the same two numbers):
+    // pk[2k] = head rA, keys 8k+ku, 8k+ku+1; pk[2k+1] = head rB, same keys
     auto load_s = [&](int t, uint32_t (&pk)[16]) -> bool {
       if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
       tc_fence_after();
-      uint32_t sreg[32];
-      tmem_ld32(lane_base + TM_S + 32 * g, sreg);
+      uint32_t s[32];
+      tmem_ld_16x256b_x8(tbase + TM_S, s);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -443,8 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         uint32_t r;
-        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(sreg[2 * c + 1])),
-            "f"(__uint_as_float(sreg[2 * c])));
+        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(s[2 * c + 1])),
+            "f"(__uint_as_float(s[2 * c])));
         pk[c] = r;
       }
       return true;
@@ -452,11 +453,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // ship this warp's block of S(t) to the peer (one 2 KB bulk copy)
     auto send = [&](int t, const uint32_t (&pk)[16]) -> bool {
       const int xb = t & 1;
-      if (!wwait(&bar->x_free[xb], ((t >> 1) & 1) ^ 1, true, 331, t)) return false;
+      if (!wwait(&bar->x_free[xb][sw], ((t >> 1) & 1) ^ 1, true, 331, t)) return false;
       const uint32_t stg = stg_base + xb * XBUF;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + uoff[q]), "r"(pk[4 * q]),
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + q * 512 + lane * 16), "r"(pk[4 * q]),
                      "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
                      : "memory");
       }
@@ -470,7 +471,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // attend, so no TMA write is still in flight when the CTA exits
     if (!wwait(&bar->q_tma, 0, false, 338, 0)) ok = false;
     if (n_tiles > 0) {
-      // Q_r row h into TMEM: this half writes dims [144g, 144g+144) = columns [72g, 72g+72)
+      // Q_r row h into TMEM (shape .32x32b: lane = head): warps of the first
+      // warpgroup write dims [0, 144) of the CTA's 288, the second [144, 288)
+      const int g = sw >> 2;
+      const int h = static_cast<int>(quarter * 32 + lane);
       uint32_t qv[72];
 #pragma unroll
       for (int m = 0; m < 18; ++m) {
@@ -485,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         qv[4 * m + 2] = v.z;
         qv[4 * m + 3] = v.w;
       }
-      const uint32_t qaddr = lane_base + TM_Q + 72 * g;
+      const uint32_t qaddr = tmem + ((quarter * 32u) << 16) + TM_Q + 72 * g;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t t16[16];
@@ -506,17 +510,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
 
     uint32_t cur[16], nxt[16];
-    if (n_tiles > 0) ok = load_s(0, cur) && send(0, cur);
+    if (n_tiles > 0) ok = ok && load_s(0, cur) && send(0, cur);
     for (int i = 0; ok && i < n_tiles; ++i) {
       // 1. next tile's partial scores go out first, so the exchange overlaps this tile's work
       if (i + 1 < n_tiles && !(load_s(i + 1, nxt) && send(i + 1, nxt))) {
         ok = false;
         break;
       }
-      // 2. the peer's partial scores of tile i
+      // 2. the peer's partial scores of tile i (this warp's own barrier)
       const int xb = i & 1;
-      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xb], XBLK);
-      if (!wwait(&bar->x_full[xb], (i >> 1) & 1, true, 332, i)) {
+      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xb][sw], XBLK);
+      if (!wwait(&bar->x_full[xb][sw], (i >> 1) & 1, true, 332, i)) {
         ok = false;
         break;
       }
@@ -525,9 +529,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       for (int q = 0; q < 4; ++q) {
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(xp[4 * q]), "=r"(xp[4 * q + 1]), "=r"(xp[4 * q + 2]), "=r"(xp[4 * q + 3])
-                     : "r"(x_base + xb * XBUF + uoff[q])
+                     : "r"(x_base + xb * XBUF + q * 512 + lane * 16)
                      : "memory");
       }
+      // sv[2c], sv[2c+1]: the pair of pk[c] (c even: head rA, c odd: head rB)
       float sv[32];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -539,44 +544,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       __syncwarp();
       // the values are in registers: the peer may refill the buffer
       if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote[xb]);
-      // 3. mask positions past the selection / padding
-      const uint32_t vbits = sValid[2 * i + g];
-      if (vbits != 0xffffffffu) {
+      // 3. mask positions past the selection / padding: key 8k + ku + e
+      const uint64_t vmask = static_cast<uint64_t>(sValid[2 * i]) | (static_cast<uint64_t>(sValid[2 * i + 1]) << 32);
+      if (vmask != ~uint64_t(0)) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (!((vbits >> c) & 1u)) sv[c] = NEG_INF;
-      }
-      // 4. row max over all 64 columns (the other half through shared memory)
-      float pm = sv[0];
+        for (int k = 0; k < 8; ++k) {
 #pragma unroll
-      for (int c = 1; c < 32; ++c) pm = fmaxf(pm, sv[c]);
-      float* red = sRed + (i & 1) * 256;     // double-buffered by tile parity
-      red[g * 128 + h] = pm;
-      mbar_arrive(&bar->red);
-      if (!wwait(&bar->red, i & 1, false, 336, i)) {
-        ok = false;
-        break;
+          for (int e = 0; e < 2; ++e) {
+            if (!((vmask >> (8 * k + ku + e)) & 1u)) {
+              sv[4 * k + e] = NEG_INF;
+              sv[4 * k + 2 + e] = NEG_INF;
+            }
+          }
+        }
       }
-      const float mz = fmaxf(pm, red[(g ^ 1) * 128 + h]) * scale;
-      const float m_new = fmaxf(m_run, mz);
-      const bool grow = m_new > m_run + 8.0f;           // true on the first finite tile
-      float alpha = 1.f;
-      if (grow) {
-        alpha = fast_exp2(m_run - m_new);                // exp2(-inf) = 0
-        m_run = m_new;
+      // 4. row maxima over the 64 columns: 16 per lane, then the lane group
+      float mA = fmaxf(sv[0], sv[1]), mB = fmaxf(sv[2], sv[3]);
+#pragma unroll
+      for (int k = 1; k < 8; ++k) {
+        mA = fmaxf(mA, fmaxf(sv[4 * k], sv[4 * k + 1]));
+        mB = fmaxf(mB, fmaxf(sv[4 * k + 2], sv[4 * k + 3]));
       }
-      const float m_ref = m_run == NEG_INF ? 0.f : m_run;
-      // 5. probabilities (fp16 pairs) and this half's row sum
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, o));
+        mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, o));
+      }
+      float alphaA = 1.f, alphaB = 1.f;
+      bool grow = false;
+      {
+        const float nA = fmaxf(m_runA, mA * scale), nB = fmaxf(m_runB, mB * scale);
+        if (nA > m_runA + 8.0f) {                      // true on the first finite tile
+          alphaA = fast_exp2(m_runA - nA);             // exp2(-inf) = 0
+          m_runA = nA;
+          grow = true;
+        }
+        if (nB > m_runB + 8.0f) {
+          alphaB = fast_exp2(m_runB - nB);
+          m_runB = nB;
+          grow = true;
+        }
+      }
+      const float refA = m_runA == NEG_INF ? 0.f : m_runA;
+      const float refB = m_runB == NEG_INF ? 0.f : m_runB;
+      // 5. probabilities (fp16 pairs, in the .16x128b order of P's columns) and row sums
       uint32_t pk[16];
-      float rs = 0.f;
+      float sA = 0.f, sB = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float pa = fast_exp2(fmaf(sv[2 * c], scale, -m_ref));
-        const float pb = fast_exp2(fmaf(sv[2 * c + 1], scale, -m_ref));
-        rs += pa + pb;
-        pk[c] = pack_half2(pa, pb);
+      for (int k = 0; k < 8; ++k) {
+        const float a0 = fast_exp2(fmaf(sv[4 * k], scale, -refA));
+        const float a1 = fast_exp2(fmaf(sv[4 * k + 1], scale, -refA));
+        const float b0 = fast_exp2(fmaf(sv[4 * k + 2], scale, -refB));
+        const float b1 = fast_exp2(fmaf(sv[4 * k + 3], scale, -refB));
+        sA += a0 + a1;
+        sB += b0 + b1;
+        pk[2 * k] = pack_half2(a0, a1);
+        pk[2 * k + 1] = pack_half2(b0, b1);
       }
-      l_run = l_run * alpha + rs;
+      l_runA = l_runA * alphaA + sA;
+      l_runB = l_runB * alphaB + sB;
       // 6. PV(i-1) must be done before P and O are touched
       if (i > 0 && !wwait(&bar->pv_done, (i - 1) & 1, false, 333, i)) {
         ok = false;
@@ -587,15 +613,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          const uint32_t oa = lane_base + TM_O + 128 * g + 32 * c;
-          tmem_ld32(oa, o);
+          tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(oa, o);
+          for (int k = 0; k < 8; ++k) {
+            o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alphaA);
+            o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alphaA);
+            o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alphaB);
+            o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alphaB);
+          }
+          tmem_st_16x256b_x8(tbase + TM_O + 64 * c, o);
         }
       }
-      tmem_st16(lane_base + TM_P + 16 * g, pk);
+      tmem_st_16x128b_x8(tbase + TM_P, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -607,48 +637,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // ---- epilogue: O / l -> bf16 (or fp32 partial) ----
     if (ok && n_tiles > 0 && !wwait(&bar->pv_done, (n_tiles - 1) & 1, false, 335, n_tiles)) ok = false;
     tc_fence_after();
-    float* lsum = sRed + 512;
-    lsum[g * 128 + h] = l_run;
-    mbar_arrive(&bar->red);
-    if (ok && !wwait(&bar->red, n_tiles & 1, false, 337, n_tiles)) ok = false;
-    const float l = lsum[h] + lsum[128 + h];            // same order in both halves
-    const bool any = n_tiles > 0 && l > 0.f;
-    const float inv_l = any ? 1.f / l : 0.f;
-    const float lse_val = any ? (m_run + __log2f(l)) * 0.69314718055994531f : NEG_INF;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      l_runA += __shfl_xor_sync(0xffffffffu, l_runA, o);
+      l_runB += __shfl_xor_sync(0xffffffffu, l_runB, o);
+    }
+    const bool anyA = n_tiles > 0 && l_runA > 0.f, anyB = n_tiles > 0 && l_runB > 0.f;
+    const float invA = anyA ? 1.f / l_runA : 0.f, invB = anyB ? 1.f / l_runB : 0.f;
+    const float lseA = anyA ? (m_runA + __log2f(l_runA)) * 0.69314718055994531f : NEG_INF;
+    const float lseB = anyB ? (m_runB + __log2f(l_runB)) * 0.69314718055994531f : NEG_INF;
+    // O chunk c (64 of the CTA's 256 value dims) of this warp's 16 heads
+    auto load_o = [&](int c, uint32_t (&o)[32]) {
+      if (n_tiles > 0) {
+        tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = 0u;
+      }
+    };
     if (p.nsplit == 1) {
       // O / l as bf16 into ring stages 0-1 (idle now) in the 128-byte-swizzled
       // layout of four [H x 64-dim] TMA boxes, then one thread stores the boxes:
-      // whole rows leave the SM instead of 16-byte pieces strided by a head row.
+      // whole rows leave the SM instead of pieces strided by a head row.
       uint8_t* sO = sKV;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld32(lane_base + TM_O + 128 * g + 32 * c, o);
-          tmem_ld_wait();
-        } else {
+        load_o(c, o);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
-        }
-        if (h < H) {
-          const int bx = 2 * g + (c >> 1), ub = (c & 1) * 4;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[8 * q + 2 * e]) * inv_l,
-                                                             __uint_as_float(o[8 * q + 2 * e + 1]) * inv_l);
-              w4[e] = *reinterpret_cast<const uint32_t*>(&v);
-            }
-            *reinterpret_cast<uint4*>(sO + bx * kQBox + h * 128 + (((ub + q) ^ (h & 7)) << 4)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int k = 0; k < 8; ++k) {
+          // dims 64c + 8k + ku, +1: box c, 16-byte unit k, byte 2*ku
+          if (hA < H) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[4 * k]) * invA,
+                                                           __uint_as_float(o[4 * k + 1]) * invA);
+            *reinterpret_cast<__nv_bfloat162*>(sO + c * kQBox + hA * 128 + ((k ^ (hA & 7)) << 4) + 2 * ku) = v;
+          }
+          if (hB < H) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[4 * k + 2]) * invB,
+                                                           __uint_as_float(o[4 * k + 3]) * invB);
+            *reinterpret_cast<__nv_bfloat162*>(sO + c * kQBox + hB * 128 + ((k ^ (hB & 7)) << 4) + 2 * ku) = v;
           }
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&bar->red);
-      const bool staged = wwait(&bar->red, (n_tiles + 1) & 1, false, 339, n_tiles);
+      const bool staged = wwait(&bar->red, 0, false, 339, n_tiles);
       if (staged && sw == 0 && lane == 0) {
 #pragma unroll
         for (int bx = 0; bx < 4; ++bx)
@@ -656,31 +690,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         bulk_commit_group();
         bulk_wait_all();
       }
-      if (rank == 0 && g == 0 && h < H && p.lse != nullptr) p.lse[static_cast<int64_t>(row) * H + h] = lse_val;
+      if (rank == 0 && (lane & 3u) == 0 && p.lse != nullptr) {
+        if (hA < H) p.lse[static_cast<int64_t>(row) * H + hA] = lseA;
+        if (hB < H) p.lse[static_cast<int64_t>(row) * H + hB] = lseB;
+      }
     } else {
-      const int64_t prow_i = (static_cast<int64_t>(row) * p.nsplit + split) * 128 + h;
-      float* orow = p.part_o + prow_i * 512 + rank * 256 + 128 * g;
+      const int64_t prow = (static_cast<int64_t>(row) * p.nsplit + split) * 128;
+      float* oA = p.part_o + (prow + hA) * 512 + rank * 256 + ku;
+      float* oB = p.part_o + (prow + hB) * 512 + rank * 256 + ku;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld32(lane_base + TM_O + 128 * g + 32 * c, o);
-          tmem_ld_wait();
-        } else {
+        load_o(c, o);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          *reinterpret_cast<float4*>(orow + c * 32 + q * 4) =
-              make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
-                          __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+        for (int k = 0; k < 8; ++k) {
+          *reinterpret_cast<float2*>(oA + 64 * c + 8 * k) =
+              make_float2(__uint_as_float(o[4 * k]) * invA, __uint_as_float(o[4 * k + 1]) * invA);
+          *reinterpret_cast<float2*>(oB + 64 * c + 8 * k) =
+              make_float2(__uint_as_float(o[4 * k + 2]) * invB, __uint_as_float(o[4 * k + 3]) * invB);
         }
       }
-      if (rank == 0 && g == 0) p.part_lse[prow_i] = lse_val;
+      if (rank == 0 && (lane & 3u) == 0) {
+        p.part_lse[prow + hA] = lseA;
+        p.part_lse[prow + hB] = lseB;
+      }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   cluster_sync();          // the peer no longer touches our shared memory
