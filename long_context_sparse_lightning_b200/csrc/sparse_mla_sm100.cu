@@ -103,7 +103,12 @@ struct Cfg {
   static constexpr int SOFT0 = NPROD + 1;
   static constexpr int THREADS = (NPROD + 1 + 8) * 32;
   static constexpr int PTHREADS = NPROD * 32;
+  // registers per thread: 128 at launch; the producer + MMA warpgroups give up
+  // 32 each so the softmax warpgroups get 160 (2 x 128 x 96 + 2 x 128 x 160 =
+  // 512 x 128)
+  static constexpr uint32_t REG_LOW = 96, REG_HIGH = 160;
 };
+static_assert(2 * 128 * Cfg::REG_LOW + 2 * 128 * Cfg::REG_HIGH == Cfg::THREADS * 128, "register split");
 static_assert(Cfg::SOFT0 % 4 == 0, "softmax warps must start a warpgroup");
 static_assert(2048 % Cfg::THREADS == 0, "index staging assumes whole warps per pass");
 static_assert(4 * kQBox + 128 * 64 <= 2 * KV_STAGE, "Q slice must fit ring stages 2-3");
@@ -260,6 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   const int n_tiles = (n_ent + kTileKeys - 1) / kTileKeys;
 
   if (warp < C::NPROD) {
+    setmaxnreg_dec<C::REG_LOW>();
     // ------------------------------------------------------------ producers --
     // Each 16-byte unit goes straight to its swizzled slot with cp.async;
     // consecutive lanes take consecutive units of a row, so one warp request
@@ -338,6 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       cp_async_wait<0>();
     }
   } else if (warp == C::MMA_WARP) {
+    setmaxnreg_dec<C::REG_LOW>();
     // ----------------------------------------------------------- MMA issuer --
     if (n_tiles > 0 && elect_one()) {
       constexpr uint32_t idesc_qk = idesc_f32acc(0, 0, 128, 64, 0, 0);     // fp16 x fp16, K-major
@@ -392,6 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       }
     }
   } else {
+    setmaxnreg_inc<C::REG_HIGH>();
     // -------------------------------------------------------------- softmax --
     // Warp sw owns 16 heads -- TMEM lanes [32q + 16*(sw/4), +16) of its lane
     // quarter q = warp % 4 -- across all 64 columns of a tile, read with the
@@ -431,12 +439,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     };
     // S(t) of this warp's 16 heads, rounded to fp16 pairs (the peer receives
     // exactly these values, so both CTAs add the same two numbers):
-    // pk[2k] = head rA, keys 8k+ku, 8k+ku+1; pk[2k+1] = head rB, same keys
-    auto load_s = [&](int t, uint32_t (&pk)[16]) -> bool {
+    // pk[2k] = head rA, keys 8k+ku, 8k+ku+1; pk[2k+1] = head rB, same keys.
+    // Split in two so the TMEM load's latency overlaps other work.
+    auto load_s_issue = [&](int t, uint32_t (&s)[32]) -> bool {
       if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
       tc_fence_after();
-      uint32_t s[32];
       tmem_ld_16x256b_x8(tbase + TM_S, s);
+      return true;
+    };
+    auto load_s_finish = [&](const uint32_t (&s)[32], uint32_t (&pk)[16]) {
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -448,7 +459,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
             "f"(__uint_as_float(s[2 * c])));
         pk[c] = r;
       }
-      return true;
     };
     // ship this warp's block of S(t) to the peer (one 2 KB bulk copy)
     auto send = [&](int t, const uint32_t (&pk)[16]) -> bool {
@@ -510,10 +520,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
 
     uint32_t cur[16], nxt[16];
-    if (n_tiles > 0) ok = ok && load_s(0, cur) && send(0, cur);
+    if (n_tiles > 0) {
+      uint32_t s0[32];
+      ok = ok && load_s_issue(0, s0);
+      if (ok) {
+        load_s_finish(s0, cur);
+        ok = send(0, cur);
+      }
+    }
     for (int i = 0; ok && i < n_tiles; ++i) {
-      // 1. next tile's partial scores go out first, so the exchange overlaps this tile's work
-      if (i + 1 < n_tiles && !(load_s(i + 1, nxt) && send(i + 1, nxt))) {
+      // 1. start loading the next tile's partial scores; they are packed and
+      //    shipped to the peer once this tile's scores are assembled
+      const bool more = i + 1 < n_tiles;
+      uint32_t snext[32];
+      if (more && !load_s_issue(i + 1, snext)) {
         ok = false;
         break;
       }
@@ -587,6 +607,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       }
       const float refA = m_runA == NEG_INF ? 0.f : m_runA;
       const float refB = m_runB == NEG_INF ? 0.f : m_runB;
+      // next tile's partial scores: wait for the TMEM load, pack, ship
+      if (more) {
+        load_s_finish(snext, nxt);
+        if (!send(i + 1, nxt)) {
+          ok = false;
+          break;
+        }
+      }
       // 5. probabilities (fp16 pairs, in the .16x128b order of P's columns) and row sums
       uint32_t pk[16];
       float sA = 0.f, sB = 0.f;
