@@ -18,27 +18,30 @@
 //   Each epilogue thread owns one key (one TMEM lane) and reads that key's 64
 //   head values of a token from its own TMEM columns, so the head sum needs no
 //   cross-thread traffic; a warp stores 32 consecutive scores (128 B).
-//   Two accumulators in TMEM ping-pong between the MMA warp and two epilogue
-//   warpgroups (group g drains buffer g).
+//   Four accumulators in TMEM (2 tokens x 64 heads each) rotate between the
+//   MMA warp and four epilogue warpgroups (group g drains buffer g): four
+//   epilogue warps per SM sub-partition keep the issue slots busy while each
+//   waits on its TMEM loads and FMA chains.
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner),
-// warps 2..9 = epilogue (two warpgroups).
+// warps 2..17 = epilogue (four warpgroups).
 #include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
+constexpr int kAccBufs = 4;                  // TMEM accumulators, one per epilogue warpgroup
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 
 template <int TOK>
 struct IdxCfg {
-  static constexpr int NG = TOK == 8 ? 2 : 1;         // accumulator groups per key tile
-  static constexpr int GTOK = TOK / NG;               // tokens per group
+  static constexpr int GTOK = TOK >= 2 ? 2 : 1;      // tokens per accumulator group
+  static constexpr int NG = TOK / GTOK;               // accumulator groups per key tile
   static constexpr int N = GTOK * 64;                 // MMA N
   static constexpr int STAGES = TOK >= 4 ? 6 : 8;
-  static constexpr int TMEM_COLS = 2 * N;             // 128, 256 or 512 (powers of two)
+  static constexpr int TMEM_COLS = kAccBufs * N;      // 256 or 512 (powers of two)
   static constexpr int BOXQ = TOK * 64 < 256 ? TOK * 64 : 256;   // q rows per TMA box
   static constexpr int Q_BYTES = TOK * 64 * 128;
   static constexpr int K_BYTES = 128 * 128;
@@ -46,7 +49,7 @@ struct IdxCfg {
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_W = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 1 + 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-byte alignment
   static_assert(OFF_K % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle-128 tiles need 1024-byte alignment");
@@ -92,8 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* q_full = bars + 2 * C::STAGES;
-  uint64_t* acc_full = q_full + 1;    // [2]
-  uint64_t* acc_empty = q_full + 3;   // [2]
+  uint64_t* acc_full = q_full + 1;               // [kAccBufs]
+  uint64_t* acc_empty = q_full + 1 + kAccBufs;    // [kAccBufs]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
 
   const uint32_t warp = warp_id();
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);   // one arrival per epilogue warp of the group
     }
@@ -169,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < C::NG; ++g) {
           const int item = it * C::NG + g;
-          const int buf = item & 1;
-          if (!mbar_wait(&acc_empty[buf], ((item >> 1) & 1) ^ 1, p.budget)) {
+          const int buf = item % kAccBufs;
+          if (!mbar_wait(&acc_empty[buf], ((item / kAccBufs) & 1) ^ 1, p.budget)) {
             report_error(p.err, kDevErrTimeout, 122, it);
             ok = false;
             break;
@@ -189,22 +192,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // --------------------------------------------------- epilogue --
-    const int ew = static_cast<int>(warp) - 2;   // 0..7
+    const int ew = static_cast<int>(warp) - 2;   // 0..15
     const int g = ew >> 2;                       // accumulator buffer this warpgroup drains
     const uint32_t quarter = warp & 3u;          // TMEM lanes this warp may access
     const int key_in_tile = static_cast<int>(quarter * 32 + lane);
     const uint32_t lane_addr = (quarter * 32u) << 16;
     const int n_items = n_tiles * C::NG;
-    for (int item = g; item < n_items; item += 2) {
+    // k_scale of this thread's key in the group's next item, fetched one item ahead
+    auto key_scale = [&](int item) {
+      const int s = (tile_begin + item / C::NG) * 128 + key_in_tile;
+      return (item < n_items && s < kv) ? __ldg(&p.k_scale[kstart + s]) : 0.f;
+    };
+    float ks_next = key_scale(g);
+    for (int item = g; item < n_items; item += kAccBufs) {
       const int it = item / C::NG;
       const int grp = item % C::NG;
-      if (!mbar_wait(&acc_full[g], (item >> 1) & 1, p.budget)) {
+      const float ks = ks_next;
+      ks_next = key_scale(item + kAccBufs);
+      if (!mbar_wait(&acc_full[g], (item / kAccBufs) & 1, p.budget)) {
         report_error(p.err, kDevErrTimeout, 130, item);
         break;
       }
       tc_fence_after();
       const int s = (tile_begin + it) * 128 + key_in_tile;
-      const float ks = s < kv ? __ldg(&p.k_scale[kstart + s]) : 0.f;
 #pragma unroll 1
       for (int tk = 0; tk < C::GTOK; ++tk) {
         const int tok = grp * C::GTOK + tk;
