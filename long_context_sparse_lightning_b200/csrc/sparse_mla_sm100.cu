@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   const int row = blockIdx.x;
   const int H = p.n_heads;
   const int S = p.nsplit;
-  for (int u = threadIdx.x; u < H * 128; u += blockDim.x) {
+  for (int u = blockIdx.y * blockDim.x + threadIdx.x; u < H * 128; u += blockDim.x * gridDim.y) {
     const int h = u >> 7, d4 = u & 127;
     const float* lse_s = p.part_lse + (static_cast<int64_t>(row) * S) * 128 + h;
     float m = __int_as_float(0xff800000);
@@ -811,12 +811,18 @@ cudaError_t launch_variant(dim3 grid, const MlaParams& p, const MlaMaps& maps, c
 }  // namespace
 
 int mla_num_splits(int total_q, int max_q_per_seq, int num_seqs, int k_sel) {
-  // fill the 74 CTA pairs of one wave about twice; keep >= 4 tiles per split
+  // A split costs a pair's fixed prologue/epilogue (~17K cycles, about five
+  // tiles of work) plus the merge, so the selection is split only when too few
+  // tokens leave most of the 74 CTA pairs of a wave idle: at 16+ tokens one pair
+  // per token is faster (measured: 64 decode tokens 91 us unsplit vs 216 us in
+  // four splits; 16 tokens 86 us vs 106 us in two).  Splits stay within one wave
+  // and keep >= 8 tiles each.
   (void)max_q_per_seq;
   (void)num_seqs;
+  if (total_q >= 16) return 1;
   const int max_tiles = (k_sel + kTileKeys - 1) / kTileKeys;
   int s = 1;
-  while (s * 2 <= max_tiles / 4 && static_cast<int64_t>(total_q) * s < 148) s *= 2;
+  while (s * 2 <= max_tiles / 8 && static_cast<int64_t>(total_q) * s * 2 * 2 <= 148) s *= 2;
   return s;
 }
 
@@ -850,7 +856,7 @@ cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_
 }
 
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream) {
-  mla_combine_kernel<<<total_q, 256, 0, stream>>>(p);
+  mla_combine_kernel<<<dim3(total_q, 16), 256, 0, stream>>>(p);   // 16 CTAs per token: few tokens, many SMs
   return cudaGetLastError();
 }
 

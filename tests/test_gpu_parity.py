@@ -49,10 +49,11 @@ def test_tiny_prefill_512_every_row():
 
 @pytest.mark.parametrize("kv,q,k_sel,H", [
     ([300, 1000, 77, 2500, 129], [5, 130, 77, 3, 1], 256, 64),     # 8-token indexer blocks, ragged tails
-    ([4000, 3100, 5000, 257], [1, 1, 1, 1], 2048, 128),            # decode: 1 token, split MLA
-    ([6000, 4100, 2049, 3000], [2, 2, 2, 2], 2048, 128),           # speculative pairs
+    ([4000, 3100, 5000, 257], [1, 1, 1, 1], 2048, 128),            # decode: 1 token, selection split in 4
+    ([6000, 4100, 2049, 3000], [2, 2, 2, 2], 2048, 128),           # speculative pairs, split in 4
     ([700, 900], [5, 4], 512, 32),                                 # 4-token indexer blocks
-    ([2100 + 37 * i for i in range(40)], [1] * 40, 2048, 128),      # decode split into 4 x 8 tiles
+    ([2100 + 37 * i for i in range(40)], [1] * 40, 2048, 128),      # 40 decode tokens, one pair each
+    ([9000, 700], [1, 1], 1024, 64),                               # 2 tokens, 16 tiles: split in 2
     ([128, 256, 384], [128, 17, 256], 64, 16),                     # exact tile multiples
 ])
 def test_ragged_batches(kv, q, k_sel, H):
