@@ -131,7 +131,11 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   const int qblocks = (b->max_q_per_seq + tok - 1) / tok;
   if (qblocks > 65535) return DSA_ERR_UNSUPPORTED;
   const int tiles = (b->max_kv_len + 127) / 128;
-  const int64_t target = int64_t(8) * 148;   // one CTA per SM (registers), ~8 waves
+  // CTAs to aim for (one per SM at a time): each CTA pays a fixed setup, so
+  // few long chunks win when there are few tokens per CTA; measured best: ~4
+  // waves with 8-token blocks (prefill), 2 with 1 token (decode), 1 with 2
+  const int64_t waves = tok >= 8 ? 4 : (tok >= 4 ? 2 : (tok == 2 ? 1 : 2));
+  const int64_t target = waves * 148;
   int tpc = tiles;
   while (tpc > 8 && static_cast<int64_t>(b->num_seqs) * qblocks * ((tiles + tpc - 1) / tpc) < target)
     tpc = (tpc + 1) / 2;
