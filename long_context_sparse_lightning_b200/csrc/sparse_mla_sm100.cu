@@ -425,17 +425,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
     float l_runA = 0.f, l_runB = 0.f;           // this lane's share of the row sums
     bool ok = true;
-    // bounded wait polled by lane 0; every lane gets the same outcome and is
-    // ordered after lane 0's acquire by the warp barrier
+    // bounded wait polled by every lane (each lane acquires for itself); the
+    // vote makes the outcome warp-uniform.  On an already completed phase this
+    // costs ~55-80 cycles, against ~280 when lane 0 polls and broadcasts.
     auto wwait = [&](uint64_t* b_, uint32_t parity, bool cluster, uint32_t site, int info) -> bool {
-      int r = 1;
-      if (lane == 0) {
-        r = cluster ? mbar_wait_cluster(b_, parity, p.budget) : mbar_wait(b_, parity, p.budget);
-        if (!r) report_error(p.err, kDevErrTimeout, site, info);
-      }
-      r = __shfl_sync(0xffffffffu, r, 0);
-      __syncwarp();
-      return r != 0;
+      const bool r = cluster ? mbar_wait_cluster(b_, parity, p.budget) : mbar_wait(b_, parity, p.budget);
+      const bool all = __all_sync(0xffffffffu, r);
+      if (!all && lane == 0) report_error(p.err, kDevErrTimeout, site, info);
+      return all;
     };
     // S(t) of this warp's 16 heads, rounded to fp16 pairs (the peer receives
     // exactly these values, so both CTAs add the same two numbers):
