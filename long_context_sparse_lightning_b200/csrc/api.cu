@@ -103,7 +103,7 @@ size_t mla_part_bytes(const dsa_batch_t* b, int k_sel) {
   const MlaSplit sp = mla_split(b, k_sel);
   if (sp.nsplit <= 1) return 0;
   const size_t rows = static_cast<size_t>(b->total_q) * sp.nsplit * 128;
-  return align_up(rows * 512 * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
+  return align_up(rows * 512 * sizeof(float), 256) + align_up(rows * 2 * sizeof(float), 256);
 }
 
 bool mla_copy(const dsa_batch_t* b, int k_sel) {

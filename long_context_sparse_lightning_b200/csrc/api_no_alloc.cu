@@ -78,7 +78,7 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   const int nsplit = dsa::mla_num_splits(b->total_q, b->max_q_per_seq, b->num_seqs, k_sel);
   const size_t rows = static_cast<size_t>(b->total_q) * nsplit * 128;
   const size_t o_bytes = nsplit > 1 ? round_up(rows * 512 * sizeof(float), 256) : 0;
-  const size_t lse_bytes = nsplit > 1 ? round_up(rows * sizeof(float), 256) : 0;
+  const size_t lse_bytes = nsplit > 1 ? round_up(rows * 2 * sizeof(float), 256) : 0;
   if (kHeader + o_bytes + lse_bytes > DSA_NO_ALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
   if (b->total_q == 0) return DSA_OK;
 

@@ -63,7 +63,7 @@ struct MlaParams {
   uint16_t* out = nullptr;            // bf16 [total_q, H, 512]
   float* lse = nullptr;               // [total_q, H] or nullptr
   float* part_o = nullptr;            // [total_q, nsplit, 128, 512] fp32 when nsplit > 1
-  float* part_lse = nullptr;          // [total_q, nsplit, 128]
+  float* part_lse = nullptr;          // [total_q, nsplit, 2 value halves, 128]
   int32_t nsplit = 1;
   int32_t keys_per_split = 0;         // multiple of 64
   uint32_t* err = nullptr;

@@ -28,14 +28,16 @@
 //              instruction and measured ~6 B/clk per SM on this pattern;
 //              16-byte cp.async from 7 warps sustains several times that.)
 //   MMA warp   S_r = Q_r . C_r^T (M=128, N=64, K=288) then O_r += P . V_r (N=256);
-//   softmax    8 warps, two per TMEM lane quarter, each half owning 32 of the 64
-//              columns: each warp ships its 2 KB of partial scores (fp16; both
-//              CTAs then add the same two rounded numbers, so S is bit-identical
-//              in both) to the peer with one bulk shared-to-shared copy, one tile
-//              ahead of its own use so the transfer overlaps a whole iteration;
-//              row max across the halves through shared memory; online softmax
-//              in log2 units with a lazily refreshed max (O rescaled in TMEM only
-//              when the max grows by more than 2^8); P stored to TMEM as fp16.
+//   softmax    8 warps, 16 heads x 64 columns each: each warp ships its 2 KB of
+//              partial scores (fp16) to the peer with one bulk shared-to-shared
+//              copy, one tile ahead of its own use so the transfer overlaps a
+//              whole iteration, and adds the peer's fp16 partial to its own fp32
+//              one; online softmax in log2 units with a lazily refreshed max (O
+//              rescaled in TMEM only when the max grows by more than 2^8); P
+//              stored to TMEM as fp16.  The two CTAs' scores differ by the fp16
+//              rounding of one partial; each CTA normalises its own value half
+//              with its own probabilities and row sums, so each half is an exact
+//              softmax average of its scores (the log-sum-exp comes per half).
 //   MMA order  Q.C^T runs two tiles ahead of P.V.
 // fp16 rather than bf16 inside the MMAs: with bf16 probabilities the rounding
 // noise costs ~1e-3 mean relative error on the bf16 output; fp16 keeps ~1e-4.
@@ -129,6 +131,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// (x, y) + the two fp16 halves of h2 (low half to x), each added in fp32 after
+// an exact widening: one mixed-precision add per value, no separate conversion.
+__device__ __forceinline__ float2 add_f32_h2(float x, float y, uint32_t h2) {
+  float rx, ry;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %3;\n\tadd.rn.f32.f16 %1, hi, %4;\n\t}"
+      : "=f"(rx), "=f"(ry)
+      : "r"(h2), "f"(x), "f"(y));
+  return make_float2(rx, ry);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -434,9 +447,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       if (!all && lane == 0) report_error(p.err, kDevErrTimeout, site, info);
       return all;
     };
-    // S(t) of this warp's 16 heads, rounded to fp16 pairs (the peer receives
-    // exactly these values, so both CTAs add the same two numbers):
-    // pk[2k] = head rA, keys 8k+ku, 8k+ku+1; pk[2k+1] = head rB, same keys.
+    // S(t) of this warp's 16 heads, kept in fp32 for this CTA and rounded to
+    // fp16 pairs for the peer: pk[2k] = head rA, keys 8k+ku, 8k+ku+1;
+    // pk[2k+1] = head rB, same keys.
     // Split in two so the TMEM load's latency overlaps other work.
     auto load_s_issue = [&](int t, uint32_t (&s)[32]) -> bool {
       if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
@@ -516,13 +529,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       if (lane == 0) mbar_arrive(&bar->q_full);
     }
 
-    uint32_t cur[16], nxt[16];
+    uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
     if (n_tiles > 0) {
-      uint32_t s0[32];
-      ok = ok && load_s_issue(0, s0);
+      uint32_t pk0[16];
+      ok = ok && load_s_issue(0, cur);
       if (ok) {
-        load_s_finish(s0, cur);
-        ok = send(0, cur);
+        load_s_finish(cur, pk0);
+        ok = send(0, pk0);
       }
     }
     for (int i = 0; ok && i < n_tiles; ++i) {
@@ -553,10 +566,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       float sv[32];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&cur[c]));
-        const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&xp[c]));
-        sv[2 * c] = a.x + bb.x;
-        sv[2 * c + 1] = a.y + bb.y;
+        const float2 v = add_f32_h2(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1]), xp[c]);
+        sv[2 * c] = v.x;
+        sv[2 * c + 1] = v.y;
       }
       __syncwarp();
       // the values are in registers: the peer may refill the buffer
@@ -606,6 +618,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       const float refB = m_runB == NEG_INF ? 0.f : m_runB;
       // next tile's partial scores: wait for the TMEM load, pack, ship
       if (more) {
+        uint32_t nxt[16];
         load_s_finish(snext, nxt);
         if (!send(i + 1, nxt)) {
           ok = false;
@@ -656,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->p_full);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) cur[c] = nxt[c];
+      for (int c = 0; c < 32; ++c) cur[c] = snext[c];
     }
 
     // ---- epilogue: O / l -> bf16 (or fp32 partial) ----
@@ -735,9 +748,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
               make_float2(__uint_as_float(o[4 * k + 2]) * invB, __uint_as_float(o[4 * k + 3]) * invB);
         }
       }
-      if (rank == 0 && (lane & 3u) == 0) {
-        p.part_lse[prow + hA] = lseA;
-        p.part_lse[prow + hB] = lseB;
+      if ((lane & 3u) == 0) {        // each value half with its own log-sum-exp
+        p.part_lse[(prow * 2 + rank * 128) + hA] = lseA;
+        p.part_lse[(prow * 2 + rank * 128) + hB] = lseB;
       }
     }
   }
@@ -766,14 +779,15 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   const int S = p.nsplit;
   for (int u = blockIdx.y * blockDim.x + threadIdx.x; u < H * 128; u += blockDim.x * gridDim.y) {
     const int h = u >> 7, d4 = u & 127;
-    const float* lse_s = p.part_lse + (static_cast<int64_t>(row) * S) * 128 + h;
+    // dims [4 d4, 4 d4 + 4) belong to value half d4 / 64, which has its own lse
+    const float* lse_s = p.part_lse + (static_cast<int64_t>(row) * S * 2 + (d4 >> 6)) * 128 + h;
     float m = __int_as_float(0xff800000);
-    for (int s = 0; s < S; ++s) m = fmaxf(m, lse_s[s * 128]);
+    for (int s = 0; s < S; ++s) m = fmaxf(m, lse_s[s * 256]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
     if (m != __int_as_float(0xff800000)) {
       for (int s = 0; s < S; ++s) {
-        const float w = __expf(lse_s[s * 128] - m);
+        const float w = __expf(lse_s[s * 256] - m);
         wsum += w;
         const float4 o = reinterpret_cast<const float4*>(
             p.part_o + ((static_cast<int64_t>(row) * S + s) * 128 + h) * 512)[d4];
