@@ -210,6 +210,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t lane = lane_id();
   const int tid = threadIdx.x;
 
+  // ---- this split's selected positions: loads first (one memory latency,
+  // overlapping the set-up below) ----
+  const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
+  constexpr int PER = (2048 + C::THREADS - 1) / C::THREADS;
+  int v[PER];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int j = tid + q * C::THREADS;
+    v[q] = (j < 2048 && j < e_count) ? __ldg(&idx_row[j]) : -1;
+  }
+
   // ---- barriers, then this CTA's Q slice by TMA into ring stages 2-3 (free
   // until the producers' third tile, which waits for q_full) ----
   uint8_t* sQ = sKV + 2 * KV_STAGE;
@@ -239,19 +250,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       tma_load_2d(sQ + c * kQBox, &maps.q_lat, &bar->q_tma, static_cast<int>(rank) * 256 + c * 64, row * H);
     tma_load_2d(sQ + 4 * kQBox, &maps.q_rope, &bar->q_tma, 512 + static_cast<int>(rank) * 32, row * H);
   }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
   __syncthreads();
 
-  // ---- this split's selected positions (invalid -> -1) and per-32 validity bits ----
-  const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
+  // ---- invalid -> -1, per-32 validity bits, the last valid slot ----
   int my_last = -1;
   {
-    constexpr int PER = (2048 + C::THREADS - 1) / C::THREADS;
-    int v[PER];
-#pragma unroll
-    for (int q = 0; q < PER; ++q) {      // all loads first: one memory latency
-      const int j = tid + q * C::THREADS;
-      v[q] = (j < 2048 && j < e_count) ? __ldg(&idx_row[j]) : -1;
-    }
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int j = tid + q * C::THREADS;
@@ -265,14 +272,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
   }
   if (my_last >= 0) atomicMax(s_last, my_last);
-
-  if (warp == C::MMA_WARP) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
   tc_fence_before();
-  cluster_sync();          // barriers of both CTAs initialised before any remote arrival
+  __syncthreads();
   tc_fence_after();
+  // Our barriers are initialised: arrive on the cluster barrier now; each role
+  // waits for the peer's arrival only before its first remote access (the
+  // softmax warps' first score exchange) or at its end, so the set-up of
+  // both CTAs overlaps the first gathers and the Q conversion.
+  cluster_arrive();
   const uint32_t tmem = *tmem_slot;
   const int n_ent = *s_last + 1;
   const int n_tiles = (n_ent + kTileKeys - 1) / kTileKeys;
@@ -356,6 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       }
       cp_async_wait<0>();
     }
+    cluster_wait();
   } else if (warp == C::MMA_WARP) {
     setmaxnreg_dec<C::REG_LOW>();
     // ----------------------------------------------------------- MMA issuer --
@@ -411,6 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
       }
     }
+    cluster_wait();
   } else {
     setmaxnreg_inc<C::REG_HIGH>();
     // -------------------------------------------------------------- softmax --
@@ -528,6 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->q_full);
     }
+    cluster_wait();          // the peer's barriers exist: exchanges may start
 
     uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
     if (n_tiles > 0) {
@@ -726,7 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         for (int bx = 0; bx < 4; ++bx)
           tma_store_2d(&maps.out, sO + bx * kQBox, static_cast<int>(rank) * 256 + bx * 64, row * H);
         bulk_commit_group();
-        bulk_wait_all();
+        bulk_wait_read_all();    // the CTA may leave once the boxes are read
       }
       if (rank == 0 && (lane & 3u) == 0 && p.lse != nullptr) {
         if (hA < H) p.lse[static_cast<int64_t>(row) * H + hA] = lseA;
