@@ -160,10 +160,10 @@ DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, co
  * cudaFree or other allocation.
  *
  *   - Batches whose partial results need more than the scratch array (more
- *     than 256 B + total_q * nsplit * 128 * 2052 B, rounded) return
+ *     than 256 B + total_q * nsplit * 128 * 2056 B, rounded) return
  *     DSA_ERR_WORKSPACE before anything is launched; use dsa_sparse_mla then.
- *     (Selections are split only for batches of fewer than 16 tokens, into at
- *     most 4 parts, so valid batches need at most ~16 MiB.)
+ *     (Selections are split only while total_q * nsplit fits 74 CTA pairs,
+ *     into at most 4 parts, so valid batches need at most ~19 MiB.)
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

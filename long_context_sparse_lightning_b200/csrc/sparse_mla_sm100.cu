@@ -832,15 +832,16 @@ cudaError_t launch_variant(dim3 grid, const MlaParams& p, const MlaMaps& maps, c
 }  // namespace
 
 int mla_num_splits(int total_q, int max_q_per_seq, int num_seqs, int k_sel) {
-  // A split costs a pair's fixed prologue/epilogue (~17K cycles, about five
-  // tiles of work) plus the merge, so the selection is split only when too few
-  // tokens leave most of the 74 CTA pairs of a wave idle: at 16+ tokens one pair
-  // per token is faster (measured: 64 decode tokens 91 us unsplit vs 216 us in
-  // four splits; 16 tokens 86 us vs 106 us in two).  Splits stay within one wave
-  // and keep >= 8 tiles each.
+  // A token's selection is split over several CTA pairs while the doubled
+  // number of pairs still fits one wave (74 pairs on 148 SMs) and every split
+  // keeps >= 8 tiles: one pair per token leaves most SMs idle on small
+  // batches, and a split's fixed cost (prologue/epilogue ~17K cycles, about
+  // five tiles, plus the log-sum-exp merge) is far below the idle time it
+  // recovers (measured, 32-tile selections: 16 tokens at 32K context 83 us
+  // unsplit vs 44 us in four splits; 8 x 2 tokens at 128K 82 vs 42 us; 64
+  // tokens stay unsplit: 91 us vs 216 us in four splits over two waves).
   (void)max_q_per_seq;
   (void)num_seqs;
-  if (total_q >= 16) return 1;
   const int max_tiles = (k_sel + kTileKeys - 1) / kTileKeys;
   int s = 1;
   while (s * 2 <= max_tiles / 8 && static_cast<int64_t>(total_q) * s * 2 * 2 <= 148) s *= 2;

@@ -77,14 +77,14 @@ def test_no_alloc_matches_workspace_entry_point_on_two_calls():
 
 
 def test_no_alloc_scratch_covers_every_split_batch():
-    # Only batches of fewer than 16 tokens have their selections split over
-    # several CTA pairs (the only case with partial results); the largest such
-    # batch must fit the fixed scratch array, so the over-size rejection stays a
-    # guard that valid batches never reach.  Sizes come from the library's own
-    # workspace rule, without touching the device.
+    # Only small batches have their selections split over several CTA pairs
+    # (total_q * nsplit within one wave of 74 pairs; the only case with partial
+    # results); the largest such batch must fit the fixed scratch array, so the
+    # over-size rejection stays a guard that valid batches never reach.  Sizes
+    # come from the library's own workspace rule, without touching the device.
     lib = dsa.library()
     worst = 0
-    for total_q in range(1, 40):
+    for total_q in range(1, 80):
         for k_sel in (64, 256, 1024, 2048):
             c = dsa._BatchC()
             c.num_seqs, c.total_q, c.max_q_per_seq, c.max_kv_len, c.total_keys = total_q, total_q, 1, 32768, total_q * 32768
