@@ -101,7 +101,10 @@ typedef struct {
 
 /* Bytes of device workspace the call `op` needs for this batch.  Returns 0
  * when the arguments are invalid.  For DSA_OP_FORWARD this includes the
- * [total_q, ld] fp32 score matrix, ld = max_kv_len rounded up to 4. */
+ * [total_q, ld] fp32 score matrix, ld = max_kv_len rounded up to 4.  For
+ * DSA_OP_TOPK (and inside DSA_OP_FORWARD) rows longer than 32768 positions
+ * with k_sel a multiple of 4 add 8 * k_sel bytes per row and 32768-position
+ * segment: the candidates of the two-phase selection. */
 DSA_API size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads);
 
 /* Indexer scores.

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -157,8 +158,15 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   return dsa::launch_indexer(tok, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// candidate buffers of the two-phase top-k (rows longer than 32768 positions)
+size_t topk_ws_bytes(const dsa_batch_t* b, int k_sel) {
+  const int segs = dsa::topk_segments(b->max_kv_len, k_sel);
+  if (segs == 0) return 0;
+  return 2 * align_up(static_cast<size_t>(b->total_q) * segs * k_sel * sizeof(float), 256);
+}
+
 dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int k_sel, int32_t* idx,
-                      uint32_t* err, cudaStream_t stream) {
+                      uint8_t* seg, uint32_t* err, cudaStream_t stream) {
   TopkParams p;
   p.cu_q = b->cu_q;
   p.kv_len = b->kv_len;
@@ -170,6 +178,13 @@ dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int
   p.num_seqs = b->num_seqs;
   p.err = err;
   p.budget = wait_budget();
+  const int segs = dsa::topk_segments(b->max_kv_len, k_sel);
+  if (segs > 0) {
+    const size_t half = align_up(static_cast<size_t>(b->total_q) * segs * k_sel * sizeof(float), 256);
+    p.seg_pos = reinterpret_cast<int32_t*>(seg);
+    p.seg_val = reinterpret_cast<float*>(seg + half);
+    p.n_seg = segs;
+  }
   return dsa::launch_topk(b->max_kv_len, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -256,15 +271,18 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, 
   if (check_batch(batch) != DSA_OK) return 0;
   switch (op) {
     case DSA_OP_INDEXER:
-    case DSA_OP_TOPK:
       return kHeaderBytes;
+    case DSA_OP_TOPK:
+      if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return 0;
+      return kHeaderBytes + topk_ws_bytes(batch, k_sel);
     case DSA_OP_SPARSE_MLA:
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
       return kHeaderBytes + mla_ws_bytes(batch, k_sel);
     case DSA_OP_FORWARD: {
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
       const size_t scores = align_up(static_cast<size_t>(batch->total_q) * forward_ld(batch) * sizeof(float), 256);
-      return kHeaderBytes + scores + mla_ws_bytes(batch, k_sel);
+      // the top-k candidates and the MLA buffers are used one after the other
+      return kHeaderBytes + scores + std::max(mla_ws_bytes(batch, k_sel), topk_ws_bytes(batch, k_sel));
     }
   }
   return 0;
@@ -292,10 +310,10 @@ dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int64_t ld_
       (ld_scores & 3) != 0)
     return DSA_ERR_INVALID_ARG;
   if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
-  if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes + topk_ws_bytes(batch, k_sel))) != DSA_OK) return s;
   if (batch->total_q == 0) return DSA_OK;
-  return run_topk(batch, scores, ld_scores, k_sel, idx, static_cast<uint32_t*>(ws),
-                  reinterpret_cast<cudaStream_t>(stream));
+  return run_topk(batch, scores, ld_scores, k_sel, idx, static_cast<uint8_t*>(ws) + kHeaderBytes,
+                  static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
@@ -330,7 +348,7 @@ dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const floa
   float* scores = reinterpret_cast<float*>(base + kHeaderBytes);
   uint8_t* part = base + kHeaderBytes + align_up(static_cast<size_t>(batch->total_q) * ld * sizeof(float), 256);
   if ((s = run_indexer(batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ld, err, st)) != DSA_OK) return s;
-  if ((s = run_topk(batch, scores, ld, k_sel, idx, err, st)) != DSA_OK) return s;
+  if ((s = run_topk(batch, scores, ld, k_sel, idx, part, err, st)) != DSA_OK) return s;
   return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, part, err, st);
 }
 

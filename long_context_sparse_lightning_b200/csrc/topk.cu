@@ -679,6 +679,122 @@ __global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) 
     select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
 }
 
+// Rows longer than the register path holds, in two phases.  Phase 1 selects
+// the top k of every kSegLen-position segment of a row (one CTA per row and
+// segment, the segment in registers) and writes the chosen positions
+// (ascending, absolute) and their scores.  A row's candidates are then the
+// concatenation of its segments' choices: all segments but the last
+// non-empty one are longer than k and give k each, so the valid candidates
+// form one prefix, ascending in position.  Phase 2 selects the top k of that
+// prefix per row; a lower candidate index is a lower position, so the tie
+// rule (equal scores: the lower position wins) carries over, and the chosen
+// indices map back to positions.  Each of the row's top k is in the top k of
+// its own segment, so the result equals a selection over the whole row.
+constexpr int kSegLen = 1024 * 32;
+
+template <int BLOCK, int EPT>
+__global__ void __launch_bounds__(BLOCK, 1) topk_segment_kernel(const TopkParams p) {
+  __shared__ TopkShared<BLOCK, BLOCK * EPT / 32> sh;
+  static_assert(BLOCK * EPT == kSegLen, "one segment in registers");
+  const int k = p.k_sel;
+  const int tid = threadIdx.x;
+  const int r = blockIdx.x, seg = blockIdx.y;
+  if (error_pending(p.err)) return;
+  int n = 0;
+  if (!row_info(p, r, n)) {
+    if (tid == 0 && seg == 0) report_error(p.err, kDevErrBounds, 203, r);
+    return;
+  }
+  const int seg0 = seg * kSegLen;
+  const int m = min(max(n - seg0, 0), kSegLen);
+  const int64_t blk = (static_cast<int64_t>(r) * p.n_seg + seg) * k;
+  int32_t* out_pos = p.seg_pos + blk;
+  float* out_val = p.seg_val + blk;
+  const float* row = p.scores + static_cast<int64_t>(r) * p.ld + seg0;
+  if (m <= k) {                            // the whole segment (or nothing)
+    for (int j = tid; j < k; j += BLOCK) {
+      out_pos[j] = j < m ? seg0 + j : -1;
+      out_val[j] = j < m ? __ldg(&row[j]) : 0.f;
+    }
+    return;
+  }
+  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
+  __syncthreads();
+  const int n_vec = (m + 3) >> 2;          // the row stride is a multiple of 4 and >= n
+  const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  float x[EPT];
+#pragma unroll
+  for (int v = 0; v < EPT / 4; ++v) {
+    const int vec = v * BLOCK + tid;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (vec < n_vec) f = __ldg(&r4[vec]);
+    x[4 * v + 0] = f.x;
+    x[4 * v + 1] = f.y;
+    x[4 * v + 2] = f.z;
+    x[4 * v + 3] = f.w;
+  }
+  auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
+  if (!select_fast<BLOCK, EPT>(sh, get4, m, n_chunks, k, __ldg(row), out_pos)) {
+    const GlobalRow<BLOCK> g{r4, n_vec};
+    select_radix<BLOCK>(sh, g, m, n_chunks, k, out_pos);
+  }
+  __syncthreads();                         // this CTA's position stores are visible to it
+  for (int j = tid; j < k; j += BLOCK) {
+    const int q = __ldcg(&out_pos[j]);     // a segment position; m > k, so never -1
+    out_val[j] = __ldg(&row[q]);
+    out_pos[j] = seg0 + q;
+  }
+}
+
+template <int BLOCK, int EPT>
+__global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p) {
+  __shared__ TopkShared<BLOCK, BLOCK * EPT / 32> sh;
+  const int k = p.k_sel;
+  const int tid = threadIdx.x;
+  const int r = blockIdx.x;
+  if (error_pending(p.err)) return;
+  int n = 0;
+  if (!row_info(p, r, n)) return;          // phase 1 reported it
+  int32_t* out = p.idx + static_cast<int64_t>(r) * k;
+  if (n <= k) {
+    fill_short_row(out, n, k, BLOCK);
+    return;
+  }
+  // valid candidates: k per full segment, then the last segment's share
+  int m = 0;
+  for (int seg = 0; seg < p.n_seg; ++seg) m += min(max(n - seg * kSegLen, 0), k);
+  const int64_t blk = static_cast<int64_t>(r) * p.n_seg * k;
+  const int32_t* cpos = p.seg_pos + blk;
+  if (m <= k) {                            // one segment's choice is the answer
+    for (int j = tid; j < k; j += BLOCK) out[j] = j < m ? __ldcg(&cpos[j]) : -1;
+    return;
+  }
+  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
+  __syncthreads();
+  const int n_vec = (m + 3) >> 2;          // k is a multiple of 4 or the tail lies inside the block
+  const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
+  const float4* c4 = reinterpret_cast<const float4*>(p.seg_val + blk);
+  float x[EPT];
+#pragma unroll
+  for (int v = 0; v < EPT / 4; ++v) {
+    const int vec = v * BLOCK + tid;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (vec < n_vec) f = __ldcg(&c4[vec]);
+    x[4 * v + 0] = f.x;
+    x[4 * v + 1] = f.y;
+    x[4 * v + 2] = f.z;
+    x[4 * v + 3] = f.w;
+  }
+  auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
+  if (!select_fast<BLOCK, EPT>(sh, get4, m, n_chunks, k, __ldcg(p.seg_val + blk), out)) {
+    const GlobalRow<BLOCK> g{c4, n_vec};
+    select_radix<BLOCK>(sh, g, m, n_chunks, k, out);
+  }
+  __syncthreads();
+  for (int j = tid; j < k; j += BLOCK) out[j] = __ldcg(&cpos[__ldcg(&out[j])]);   // candidate -> position
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -704,10 +820,23 @@ cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+int topk_segments(int max_kv_len, int k_sel) {
+  // candidate blocks of k floats must keep float4 alignment
+  if (max_kv_len <= kSegLen || k_sel < 1 || (k_sel & 3) != 0) return 0;
+  const int segs = (max_kv_len + kSegLen - 1) / kSegLen;
+  return static_cast<int64_t>(segs) * k_sel <= kSegLen ? segs : 0;   // phase 2 holds the candidates
+}
+
 cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream) {
   if (p.total_q <= 0) return cudaSuccess;
   if (max_kv_len <= 256 * 32) return launch_reg<256, 32, 2>(p, stream);
   if (max_kv_len <= 1024 * 32) return launch_reg<1024, 32, 1>(p, stream);
+  const int segs = topk_segments(max_kv_len, p.k_sel);
+  if (segs > 0 && p.seg_pos != nullptr && p.seg_val != nullptr && p.n_seg == segs) {
+    topk_segment_kernel<1024, 32><<<dim3(p.total_q, segs), 1024, 0, stream>>>(p);
+    topk_merge_kernel<1024, 32><<<p.total_q, 1024, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   topk_stream_kernel<1024><<<p.total_q, 1024, 0, stream>>>(p);
   return cudaGetLastError();
 }

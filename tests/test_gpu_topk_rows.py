@@ -97,3 +97,20 @@ def test_crowded_and_tied_rows(L):
 def test_small_k(k):
     got, exp = _run([20000, 900, 6000], [2, 3, 2], normal, k, seed=k)
     _assert_equal(got, exp)
+
+
+@pytest.mark.parametrize("kv,q", [([131072, 70000], [2, 2]), ([65536 + 100, 32768 + 5], [1, 2])])
+def test_rows_over_32768_in_segments(kv, q):
+    # rows longer than one register row go through per-segment selections and
+    # a merge; a last segment shorter than k contributes all its positions
+    got, exp = _run(kv, q, normal, 2048, seed=kv[0] % 97)
+    _assert_equal(got, exp)
+
+
+@pytest.mark.parametrize("k", [7, 300, 2048])
+def test_long_rows_mixed_with_short_ones(k):
+    # one batch of short, register-sized and long rows; k = 7 (not a multiple
+    # of 4) takes the single-CTA path for the long rows, the others the segments
+    kv = [40000, 100, 33000, 2049, 90000]
+    got, exp = _run(kv, [2, 1, 1, 1, 1], normal, k, seed=k + 3)
+    _assert_equal(got, exp)
