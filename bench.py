@@ -352,7 +352,9 @@ def main():
     # ---- per-stage device time (same stream, CUDA events between the launches) ----
     ld = ((b.max_kv_len + 3) // 4) * 4
     scores = torch.empty((b.total_q, ld), dtype=torch.float32, device=dev)
-    ws_s = dsa.workspace(dsa.OP_SPARSE_MLA, batch, k, H, device=dev)
+    # one workspace for the three standalone stages: the largest of their sizes
+    ws_op = max((dsa.OP_TOPK, dsa.OP_SPARSE_MLA), key=lambda op: dsa.workspace_size(op, batch, k, H))
+    ws_s = dsa.workspace(ws_op, batch, k, H, device=dev)
     st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for i in range(args.warmup + args.steps):
         flush.fill_(float(i))

@@ -160,9 +160,9 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
 
 // candidate buffers of the two-phase top-k (rows longer than 32768 positions)
 size_t topk_ws_bytes(const dsa_batch_t* b, int k_sel) {
-  const int segs = dsa::topk_segments(b->max_kv_len, k_sel);
-  if (segs == 0) return 0;
-  return 2 * align_up(static_cast<size_t>(b->total_q) * segs * k_sel * sizeof(float), 256);
+  const dsa::TopkSegments t = dsa::topk_segments(b->max_kv_len, k_sel, b->total_q);
+  if (t.segs == 0) return 0;
+  return 2 * align_up(static_cast<size_t>(b->total_q) * t.segs * k_sel * sizeof(float), 256);
 }
 
 dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int k_sel, int32_t* idx,
@@ -178,12 +178,13 @@ dsa_status_t run_topk(const dsa_batch_t* b, const float* scores, int64_t ld, int
   p.num_seqs = b->num_seqs;
   p.err = err;
   p.budget = wait_budget();
-  const int segs = dsa::topk_segments(b->max_kv_len, k_sel);
-  if (segs > 0) {
-    const size_t half = align_up(static_cast<size_t>(b->total_q) * segs * k_sel * sizeof(float), 256);
+  const dsa::TopkSegments t = dsa::topk_segments(b->max_kv_len, k_sel, b->total_q);
+  if (t.segs > 0) {
+    const size_t half = align_up(static_cast<size_t>(b->total_q) * t.segs * k_sel * sizeof(float), 256);
     p.seg_pos = reinterpret_cast<int32_t*>(seg);
     p.seg_val = reinterpret_cast<float*>(seg + half);
-    p.n_seg = segs;
+    p.n_seg = t.segs;
+    p.seg_len = t.len;
   }
   return dsa::launch_topk(b->max_kv_len, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

@@ -44,15 +44,21 @@ struct TopkParams {
   int32_t num_seqs;
   uint32_t* err;
   long long budget;       // clock64 cycles a bulk-copy wait may take
-  // rows longer than 32768 positions, two-phase path (topk_segments > 0):
-  // [total_q, n_seg, k_sel] candidate positions and their scores
+  // two-phase path (topk_segments(...).segs > 0): n_seg segments of seg_len
+  // positions per row; [total_q, n_seg, k_sel] candidate positions and scores
   int32_t* seg_pos = nullptr;
   float* seg_val = nullptr;
   int32_t n_seg = 0;
+  int32_t seg_len = 0;
 };
 
-// Segments of the two-phase path for this row length and k (0: not used).
-int topk_segments(int max_kv_len, int k_sel);
+// Two-phase top-k plan: rows longer than 32768 positions are selected per
+// segment and then merged.  segs == 0: the single-pass kernels.
+struct TopkSegments {
+  int segs;
+  int len;
+};
+TopkSegments topk_segments(int max_kv_len, int k_sel, int total_q);
 cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream);
 
 // ------------------------------------------------------------- sparse MLA --

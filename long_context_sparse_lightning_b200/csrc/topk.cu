@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) 
 }
 
 // Rows longer than the register path holds, in two phases.  Phase 1 selects
-// the top k of every kSegLen-position segment of a row (one CTA per row and
+// the top k of every seg_len-position segment of a row (one CTA per row and
 // segment, the segment in registers) and writes the chosen positions
 // (ascending, absolute) and their scores.  A row's candidates are then the
 // concatenation of its segments' choices: all segments but the last
@@ -690,12 +690,13 @@ __global__ void __launch_bounds__(BLOCK) topk_stream_kernel(const TopkParams p) 
 // rule (equal scores: the lower position wins) carries over, and the chosen
 // indices map back to positions.  Each of the row's top k is in the top k of
 // its own segment, so the result equals a selection over the whole row.
-constexpr int kSegLen = 1024 * 32;
+constexpr int kSegLen = 1024 * 32;        // longest segment: one register row
 
 template <int BLOCK, int EPT>
 __global__ void __launch_bounds__(BLOCK, 1) topk_segment_kernel(const TopkParams p) {
   __shared__ TopkShared<BLOCK, BLOCK * EPT / 32> sh;
   static_assert(BLOCK * EPT == kSegLen, "one segment in registers");
+  const int seg_len = p.seg_len;           // <= kSegLen, a multiple of 4
   const int k = p.k_sel;
   const int tid = threadIdx.x;
   const int r = blockIdx.x, seg = blockIdx.y;
@@ -705,8 +706,8 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_segment_kernel(const TopkParams
     if (tid == 0 && seg == 0) report_error(p.err, kDevErrBounds, 203, r);
     return;
   }
-  const int seg0 = seg * kSegLen;
-  const int m = min(max(n - seg0, 0), kSegLen);
+  const int seg0 = seg * seg_len;
+  const int m = min(max(n - seg0, 0), seg_len);
   const int64_t blk = (static_cast<int64_t>(r) * p.n_seg + seg) * k;
   int32_t* out_pos = p.seg_pos + blk;
   float* out_val = p.seg_val + blk;
@@ -763,7 +764,7 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p
   }
   // valid candidates: k per full segment, then the last segment's share
   int m = 0;
-  for (int seg = 0; seg < p.n_seg; ++seg) m += min(max(n - seg * kSegLen, 0), k);
+  for (int seg = 0; seg < p.n_seg; ++seg) m += min(max(n - seg * p.seg_len, 0), k);
   const int64_t blk = static_cast<int64_t>(r) * p.n_seg * k;
   const int32_t* cpos = p.seg_pos + blk;
   if (m <= k) {                            // one segment's choice is the answer
@@ -820,19 +821,27 @@ cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-int topk_segments(int max_kv_len, int k_sel) {
+TopkSegments topk_segments(int max_kv_len, int k_sel, int total_q) {
+  TopkSegments t{0, 0};
   // candidate blocks of k floats must keep float4 alignment
-  if (max_kv_len <= kSegLen || k_sel < 1 || (k_sel & 3) != 0) return 0;
+  if (k_sel < 1 || (k_sel & 3) != 0 || total_q < 1 || max_kv_len <= kSegLen) return t;
+  // as few segments as register rows allow, of equal length.  (Splitting rows
+  // that fit one register row, to put more CTAs on few rows, was slower:
+  // 64 rows of 16K-32K positions 24 us in one CTA per row, 34 us in halves;
+  // nor did 9 segments beat 4 on 16 rows of 128K: 38 us each.)
   const int segs = (max_kv_len + kSegLen - 1) / kSegLen;
-  return static_cast<int64_t>(segs) * k_sel <= kSegLen ? segs : 0;   // phase 2 holds the candidates
+  if (static_cast<int64_t>(segs) * k_sel > kSegLen) return t;        // phase 2 holds the candidates
+  t.segs = segs;
+  t.len = (((max_kv_len + segs - 1) / segs) + 3) & ~3;
+  return t;
 }
 
 cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream) {
   if (p.total_q <= 0) return cudaSuccess;
-  if (max_kv_len <= 256 * 32) return launch_reg<256, 32, 2>(p, stream);
-  if (max_kv_len <= 1024 * 32) return launch_reg<1024, 32, 1>(p, stream);
-  const int segs = topk_segments(max_kv_len, p.k_sel);
-  if (segs > 0 && p.seg_pos != nullptr && p.seg_val != nullptr && p.n_seg == segs) {
+  if (p.n_seg == 0 && max_kv_len <= 256 * 32) return launch_reg<256, 32, 2>(p, stream);
+  if (p.n_seg == 0 && max_kv_len <= 1024 * 32) return launch_reg<1024, 32, 1>(p, stream);
+  const int segs = p.n_seg;
+  if (segs > 0 && p.seg_pos != nullptr && p.seg_val != nullptr && p.seg_len > 0) {
     topk_segment_kernel<1024, 32><<<dim3(p.total_q, segs), 1024, 0, stream>>>(p);
     topk_merge_kernel<1024, 32><<<p.total_q, 1024, 0, stream>>>(p);
     return cudaGetLastError();
