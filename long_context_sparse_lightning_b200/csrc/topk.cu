@@ -131,6 +131,22 @@ __device__ __forceinline__ void for_range(int v0, int v1, Fn&& fn) {
   }
 }
 
+// Register rows (EPT > 0) hold -inf at positions >= n: no score reaches the
+// finite histogram bound there, so only the range pass needs the row length.
+__device__ __forceinline__ float4 load_padded(const float4* src, int vec, int n_vec, int n, bool cg) {
+  const float NI = __int_as_float(0xff800000);
+  if (vec >= n_vec) return make_float4(NI, NI, NI, NI);
+  float4 f = cg ? __ldcg(&src[vec]) : src[vec];
+  const int p0 = vec * 4;
+  if (p0 + 4 > n) {
+    if (p0 + 1 > n) f.x = NI;
+    if (p0 + 2 > n) f.y = NI;
+    if (p0 + 3 > n) f.z = NI;
+    f.w = NI;
+  }
+  return f;
+}
+
 // max / min that return NaN when either input is NaN
 __device__ __forceinline__ float max_nan(float a, float b) {
   float r;
@@ -245,7 +261,7 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
       const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (pos_of(v, c) < n && e[c] >= lo) atomicAdd(&sh.hist[bin_of(e[c])], 1u);
+        if ((EPT > 0 || pos_of(v, c) < n) && e[c] >= lo) atomicAdd(&sh.hist[bin_of(e[c])], 1u);
     });
     __syncthreads();
     // ---- bin b* with count(bins above) < k <= count(bins at or above) ----
@@ -292,7 +308,7 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
       uint32_t cs = 0, cb = 0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int b = (pos_of(v, c) < n && e[c] >= lo) ? bin_of(e[c]) : -1;
+        const int b = ((EPT > 0 || pos_of(v, c) < n) && e[c] >= lo) ? bin_of(e[c]) : -1;
         cs |= static_cast<uint32_t>(b > bstar) << c;
         cb |= static_cast<uint32_t>(b == bstar) << c;
       }
@@ -629,9 +645,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
     const float4* b4 = reinterpret_cast<const float4*>(buf);
 #pragma unroll
     for (int v = 0; v < EPT / 4; ++v) {
-      const int vec = v * BLOCK + tid;
-      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (vec < n_vec) f = b4[vec];
+      const float4 f = load_padded(b4, v * BLOCK + tid, n_vec, n, false);
       x[4 * v + 0] = f.x;
       x[4 * v + 1] = f.y;
       x[4 * v + 2] = f.z;
@@ -727,9 +741,7 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_segment_kernel(const TopkParams
   float x[EPT];
 #pragma unroll
   for (int v = 0; v < EPT / 4; ++v) {
-    const int vec = v * BLOCK + tid;
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (vec < n_vec) f = __ldg(&r4[vec]);
+    const float4 f = load_padded(r4, v * BLOCK + tid, n_vec, m, false);
     x[4 * v + 0] = f.x;
     x[4 * v + 1] = f.y;
     x[4 * v + 2] = f.z;
@@ -779,9 +791,7 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p
   float x[EPT];
 #pragma unroll
   for (int v = 0; v < EPT / 4; ++v) {
-    const int vec = v * BLOCK + tid;
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (vec < n_vec) f = __ldcg(&c4[vec]);
+    const float4 f = load_padded(c4, v * BLOCK + tid, n_vec, m, true);
     x[4 * v + 0] = f.x;
     x[4 * v + 1] = f.y;
     x[4 * v + 2] = f.z;
