@@ -55,6 +55,8 @@ def test_tiny_prefill_512_every_row():
     ([2100 + 37 * i for i in range(40)], [1] * 40, 2048, 128),      # 40 decode tokens, one pair each
     ([9000, 700], [1, 1], 1024, 64),                               # 2 tokens, 16 tiles: split in 2
     ([128, 256, 384], [128, 17, 256], 64, 16),                     # exact tile multiples
+    ([3000], [100], 2048, 64),                                     # one sequence over more tokens than CTA pairs
+    ([5000], [80], 1024, 128),                                     # the same with 16-tile selections
 ])
 def test_ragged_batches(kv, q, k_sel, H):
     x = make_inputs(custom_workload("ragged", kv, q, k_sel=k_sel, n_heads=H), seed=11)
