@@ -55,6 +55,24 @@ struct IdxCfg {
   static_assert(OFF_K % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle-128 tiles need 1024-byte alignment");
 };
 
+// Two fp32 values as one 64-bit register pair (low half first) and a packed
+// fma: each lane computes fma.rn.f32 of its pair of elements.
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return make_float2(lo, hi);
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -223,25 +241,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(taddr, ra);
         tmem_ld32(taddr + 32, rb);
         tmem_ld_wait();
-        const float4* w4 = reinterpret_cast<const float4*>(sW + tok * 64);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        // four running sums (heads j mod 4) kept as two f32x2 pairs: each
+        // lane of fma.rn.f32x2 is the fp32 fma of the scalar form, so the
+        // sums are bit-identical to it, in half the FMA instructions
+        const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(sW + tok * 64);
+        unsigned long long a01 = 0ull, a23 = 0ull;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 wv = w4[j];
-          a0 = fmaf(wv.x, fmaxf(__uint_as_float(ra[4 * j + 0]), 0.f), a0);
-          a1 = fmaf(wv.y, fmaxf(__uint_as_float(ra[4 * j + 1]), 0.f), a1);
-          a2 = fmaf(wv.z, fmaxf(__uint_as_float(ra[4 * j + 2]), 0.f), a2);
-          a3 = fmaf(wv.w, fmaxf(__uint_as_float(ra[4 * j + 3]), 0.f), a3);
+          const ulonglong2 wv = w2[j];
+          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(ra[4 * j + 0]), 0.f),
+                                  fmaxf(__uint_as_float(ra[4 * j + 1]), 0.f)), a01);
+          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(ra[4 * j + 2]), 0.f),
+                                  fmaxf(__uint_as_float(ra[4 * j + 3]), 0.f)), a23);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 wv = w4[8 + j];
-          a0 = fmaf(wv.x, fmaxf(__uint_as_float(rb[4 * j + 0]), 0.f), a0);
-          a1 = fmaf(wv.y, fmaxf(__uint_as_float(rb[4 * j + 1]), 0.f), a1);
-          a2 = fmaf(wv.z, fmaxf(__uint_as_float(rb[4 * j + 2]), 0.f), a2);
-          a3 = fmaf(wv.w, fmaxf(__uint_as_float(rb[4 * j + 3]), 0.f), a3);
+          const ulonglong2 wv = w2[8 + j];
+          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(rb[4 * j + 0]), 0.f),
+                                  fmaxf(__uint_as_float(rb[4 * j + 1]), 0.f)), a01);
+          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(rb[4 * j + 2]), 0.f),
+                                  fmaxf(__uint_as_float(rb[4 * j + 3]), 0.f)), a23);
         }
-        const float acc = (a0 + a1) + (a2 + a3);
+        const float2 s01 = unpack2(a01), s23 = unpack2(a23);
+        const float acc = (s01.x + s01.y) + (s23.x + s23.y);
         if (tok < ntok && s <= t_first + tok) {
           p.scores[static_cast<int64_t>(row0 + tok) * p.ld + s] = acc * ks;
         }
