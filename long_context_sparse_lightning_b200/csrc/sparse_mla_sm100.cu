@@ -144,6 +144,28 @@ __device__ __forceinline__ float2 add_f32_h2(float x, float y, uint32_t h2) {
   return make_float2(rx, ry);
 }
 
+// f32x2 register pairs (low element first) and their packed fma / add
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -636,21 +658,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
       }
       // 5. probabilities (fp16 pairs, in the .16x128b order of P's columns) and row sums
+      // (exponent arguments and row sums on f32x2 pairs: half the FMA/add
+      // instructions; each lane is the fp32 operation of the scalar form)
       uint32_t pk[16];
-      float sA = 0.f, sB = 0.f;
+      const uint64_t sc2 = pack_f32x2(scale, scale);
+      const uint64_t nA2 = pack_f32x2(-refA, -refA), nB2 = pack_f32x2(-refB, -refB);
+      uint64_t sA2 = 0ull, sB2 = 0ull;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float a0 = fast_exp2(fmaf(sv[4 * k], scale, -refA));
-        const float a1 = fast_exp2(fmaf(sv[4 * k + 1], scale, -refA));
-        const float b0 = fast_exp2(fmaf(sv[4 * k + 2], scale, -refB));
-        const float b1 = fast_exp2(fmaf(sv[4 * k + 3], scale, -refB));
-        sA += a0 + a1;
-        sB += b0 + b1;
+        const float2 xa = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * k], sv[4 * k + 1]), sc2, nA2));
+        const float2 xb = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * k + 2], sv[4 * k + 3]), sc2, nB2));
+        const float a0 = fast_exp2(xa.x), a1 = fast_exp2(xa.y);
+        const float b0 = fast_exp2(xb.x), b1 = fast_exp2(xb.y);
+        sA2 = add_f32x2(sA2, pack_f32x2(a0, a1));
+        sB2 = add_f32x2(sB2, pack_f32x2(b0, b1));
         pk[2 * k] = pack_half2(a0, a1);
         pk[2 * k + 1] = pack_half2(b0, b1);
       }
-      l_runA = l_runA * alphaA + sA;
-      l_runB = l_runB * alphaB + sB;
+      const float2 sa = unpack_f32x2(sA2), sb = unpack_f32x2(sB2);
+      l_runA = l_runA * alphaA + (sa.x + sa.y);
+      l_runB = l_runB * alphaB + (sb.x + sb.y);
       // 6. PV(i-1) must be done before P and O are touched
       if (i > 0 && !wwait(&bar->pv_done, (i - 1) & 1, false, 333, i)) {
         ok = false;
