@@ -347,7 +347,7 @@ def main():
         pg.all_reduce(tt, op=pg.ReduceOp.MAX)
         sec = float(tt.item())
     value = world * b.total_q * args.steps / sec
-    launches_per_step = 3 + (1 if dsa_nsplit(b, k) > 1 else 0)
+    launches_per_step = dsa.forward_launches(batch, k, H)
 
     # ---- per-stage device time (same stream, CUDA events between the launches) ----
     ld = ((b.max_kv_len + 3) // 4) * 4
@@ -464,15 +464,6 @@ def main():
             "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
     print(json.dumps(line), flush=True)
     return 0
-
-
-def dsa_nsplit(b, k_sel):
-    # mirrors the library's split heuristic for the launch count (>= 4 tiles per split, fill 148 SMs)
-    tiles = (k_sel + 63) // 64
-    s = 1
-    while s * 2 <= tiles // 4 and b.total_q * s < 148:
-        s *= 2
-    return s
 
 
 if __name__ == "__main__":

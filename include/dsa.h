@@ -189,6 +189,13 @@ DSA_API dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* batch, const voi
  * receive the kernel site id and detail recorded with the error. */
 DSA_API dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info);
 
+/* Kernel launches one dsa_forward call makes for this batch: the indexer, the
+ * top-k (two for rows longer than 32768 positions with k_sel a multiple of 4),
+ * the fp16 copy of the latent cache when the selections reuse its rows often,
+ * the sparse MLA, and the merge of split selections.  0 when the arguments are
+ * invalid.  Host-only; for accounting and profiling. */
+DSA_API int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads);
+
 /* Static description of a status code. */
 DSA_API const char* dsa_status_string(dsa_status_t status);
 

@@ -46,6 +46,7 @@ EXPORTS = [
     "dsa_check_device_error",
     "dsa_status_string",
     "dsa_version",
+    "dsa_forward_launches",
 ]
 
 
@@ -99,6 +100,8 @@ def _lib():
         lib.dsa_status_string.restype = ctypes.c_char_p
         lib.dsa_version.argtypes = []
         lib.dsa_version.restype = I32
+        lib.dsa_forward_launches.argtypes = [BP, I32, I32]
+        lib.dsa_forward_launches.restype = I32
         _LIB = lib
     return _LIB
 
@@ -213,6 +216,11 @@ def check_device_error(ws, stream=None):
         err = DSAError(st, f"device error (site {site.value}, info {info.value})")
         err.site, err.info = site.value, info.value
         raise err
+
+
+def forward_launches(batch: Batch, k_sel: int, n_heads: int) -> int:
+    """Kernel launches one dsa_forward call makes for this batch (host only)."""
+    return int(_lib().dsa_forward_launches(batch.ref, k_sel, n_heads))
 
 
 def version() -> int:

@@ -353,6 +353,18 @@ dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const floa
   return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, part, err, st);
 }
 
+int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads) {
+  if (check_batch(batch) != DSA_OK) return 0;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
+  if (batch->total_q == 0) return 0;
+  int32_t n = 1;                                                             // indexer
+  n += dsa::topk_segments(batch->max_kv_len, k_sel, batch->total_q).segs > 0 ? 2 : 1;
+  if (mla_copy(batch, k_sel)) n += 1;                                        // fp16 latent copy
+  n += 1;                                                                    // sparse MLA
+  if (mla_split(batch, k_sel).nsplit > 1) n += 1;                            // merge
+  return n;
+}
+
 dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info) {
   if (ws == nullptr) return DSA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

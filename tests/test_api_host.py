@@ -66,6 +66,20 @@ def test_workspace_sizes():
     assert lib.dsa_workspace_size(dsa.OP_FORWARD, ctypes.byref(long), 2048, 128) >= 256 + extra
 
 
+def test_forward_launch_counts():
+    lib = dsa.library()
+    # short rows, few gathers per cache row: indexer, top-k, sparse MLA
+    c = _host_batch()
+    assert lib.dsa_forward_launches(ctypes.byref(c), 64, 16) == 3
+    # one long-context sequence of many queries: + the fp16 latent copy
+    pre = _host_batch(B=1, total_q=4096, max_q=4096, max_kv=32768, total_keys=32768)
+    assert lib.dsa_forward_launches(ctypes.byref(pre), 2048, 128) == 4
+    # a few decode tokens at 128K: two-phase top-k and split selections + merge
+    dec = _host_batch(B=8, total_q=16, max_q=2, max_kv=131072, total_keys=8 * 131072)
+    assert lib.dsa_forward_launches(ctypes.byref(dec), 2048, 128) == 5
+    assert lib.dsa_forward_launches(ctypes.byref(dec), 4096, 128) == 0      # k_sel too large
+
+
 def test_rejections_happen_before_any_launch():
     lib = dsa.library()
     c = _host_batch()
