@@ -238,6 +238,23 @@ def dist_setup(args):
     return world, rank, local
 
 
+def slowest_rank(sec, pg, device):
+    """The largest of the ranks' elapsed times (every rank gets it); `sec` as is
+    without a process group.  Multi-GPU numbers are timed as the max over ranks."""
+    if pg is None:
+        return sec
+    import torch
+    t = torch.tensor([float(sec)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, rows_per_rank, steps, slowest_sec):
+    """Query tokens/s of all ranks together: every rank runs its own replica of
+    the workload (weak scaling), so the job ends with the slowest rank."""
+    return world * rows_per_rank * steps / slowest_sec
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -341,12 +358,8 @@ def main():
     if pg:
         pg.barrier()
     dsa.check_device_error(ws)
-    sec = sum(a.elapsed_time(c) for a, c in ev) / 1e3
-    if pg:
-        tt = torch.tensor([sec], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        sec = float(tt.item())
-    value = world * b.total_q * args.steps / sec
+    sec = slowest_rank(sum(a.elapsed_time(c) for a, c in ev) / 1e3, pg, dev)
+    value = whole_job_rate(world, b.total_q, args.steps, sec)
     launches_per_step = dsa.forward_launches(batch, k, H)
 
     # ---- per-stage device time (same stream, CUDA events between the launches) ----
@@ -426,12 +439,8 @@ def main():
     torch.cuda.synchronize()
     for _, _, _, wsj in sets:
         dsa.check_device_error(wsj)
-    e2e_sec = e_start.elapsed_time(e_end) / 1e3
-    if pg:
-        tt = torch.tensor([e2e_sec], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e2e_sec = float(tt.item())
-    e2e_value = world * b.total_q * args.steps / e2e_sec
+    e2e_sec = slowest_rank(e_start.elapsed_time(e_end) / 1e3, pg, dev)
+    e2e_value = whole_job_rate(world, b.total_q, args.steps, e2e_sec)
 
     if pg:
         pg.barrier()
