@@ -905,7 +905,8 @@ cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_
 }
 
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream) {
-  mla_combine_kernel<<<dim3(total_q, 16), 256, 0, stream>>>(p);   // 16 CTAs per token: few tokens, many SMs
+  // 64 CTAs per token: few tokens, many SMs, one unit of (head, 4 dims) per thread
+  mla_combine_kernel<<<dim3(total_q, 64), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -99,10 +99,12 @@ def test_small_k(k):
     _assert_equal(got, exp)
 
 
-@pytest.mark.parametrize("kv,q", [([131072, 70000], [2, 2]), ([65536 + 100, 32768 + 5], [1, 2])])
+@pytest.mark.parametrize("kv,q", [([131072, 70000], [2, 2]), ([65536 + 100, 32768 + 5], [1, 2]),
+                                  ([150000, 40000], [1, 1])])
 def test_rows_over_32768_in_segments(kv, q):
     # rows longer than one register row go through per-segment selections and
-    # a merge; a last segment shorter than k contributes all its positions
+    # a merge (150000 positions make 5 segments); a last segment shorter than k
+    # contributes all its positions
     got, exp = _run(kv, q, normal, 2048, seed=kv[0] % 97)
     _assert_equal(got, exp)
 
