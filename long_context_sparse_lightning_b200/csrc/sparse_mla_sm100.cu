@@ -23,8 +23,9 @@
 //   gather     7 producer warps copy each row's 16-byte units with cp.async
 //              straight into their swizzled slots, from an fp16 copy of the
 //              latent cache (prefill: rows are reused across many tokens) or
-//              from the bf16 cache with an in-place conversion to fp16
-//              (decode); 4-stage ring.  (TMA gather4 moves 4 rows x 128 B per
+//              from the bf16 cache (decode: Q.C^T then runs in bf16 on the
+//              tile as it landed, and only afterwards do the producers convert
+//              its value part to fp16 in place for P.V); 4-stage ring.  (TMA gather4 moves 4 rows x 128 B per
 //              instruction and measured ~6 B/clk per SM on this pattern;
 //              16-byte cp.async from 7 warps sustains several times that.)
 //   MMA warp   S_r = Q_r . C_r^T (M=128, N=64, K=288) then O_r += P . V_r (N=256);
@@ -90,6 +91,8 @@ struct Bars {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
+  uint64_t qk_done[kStages];   // bf16 source: Q.C^T of the stage's tile has read it (MMA commit)
+  uint64_t v_full[kStages];    // bf16 source: the stage's value part converted to fp16 in place
   uint64_t s_full, s_empty;
   uint64_t x_full[2][8], x_free[2][8];   // per buffer and softmax warp
   uint64_t p_full, pv_done;
@@ -189,7 +192,8 @@ __device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
 }
 
 // FP16_SRC: p.kv is an fp16 copy of the latent cache (rows land ready for the
-// MMAs); otherwise p.kv is the bf16 cache and producers convert in place.
+// MMAs); otherwise p.kv is the bf16 cache: Q.C^T runs in bf16 and the producers
+// convert the value part in place between Q.C^T and P.V.
 template <bool FP16_SRC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     sparse_mla_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
@@ -253,6 +257,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->kv_full[s], C::NPROD);
       mbar_init(&bar->kv_empty[s], 1);
+      mbar_init(&bar->qk_done[s], 1);
+      mbar_init(&bar->v_full[s], C::NPROD);
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_empty, 8);
@@ -354,19 +360,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         cp_async_commit();
       };
       auto land = [&](int tile) {
-        if constexpr (!FP16_SRC) {
-          uint8_t* base = sKV + (tile % kStages) * KV_STAGE;
-#pragma unroll
-          for (int m = 0; m < UPT; ++m) {
-            if (mine(m)) {
-              uint4* q = reinterpret_cast<uint4*>(base + soff[m]);
-              *q = cvt_unit(*q);
-            }
-          }
-        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->kv_full[tile % kStages]);
+      };
+      // bf16 source: Q.C^T reads the tile as bf16 (exact products, like fp16);
+      // once it has, the value part (units 0..31) becomes fp16 in place for
+      // P.V, off the path from the gather to the scores
+      auto convert = [&](int tile) {
+        if constexpr (!FP16_SRC) {
+          const int st = tile % kStages;
+          if (ok && !mbar_wait(&bar->qk_done[st], (tile / kStages) & 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 313, tile);
+            ok = false;
+          }
+          if (ok) {
+            uint8_t* base = sKV + st * KV_STAGE;
+#pragma unroll
+            for (int m = 0; m < UPT; ++m) {
+              if (mine(m) && soff[m] < static_cast<uint32_t>(KV_ROPE)) {   // a value unit
+                uint4* q = reinterpret_cast<uint4*>(base + soff[m]);
+                *q = cvt_unit(*q);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->v_full[st]);
+        }
       };
       // land tile i before waiting for tile i+2's ring slot: that slot is
       // freed by P.V of tile i-2, which runs after Q.C^T of tile i, which
@@ -381,8 +402,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
         if (!ok) break;
         land(i);
+        if (i > 0) convert(i - 1);
         if (i + 2 < n_tiles) issue(i + 2);
       }
+      if (ok) convert(n_tiles - 1);
       cp_async_wait<0>();
     }
     cluster_wait();
@@ -390,7 +413,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     setmaxnreg_dec<C::REG_LOW>();
     // ----------------------------------------------------------- MMA issuer --
     if (n_tiles > 0 && elect_one()) {
-      constexpr uint32_t idesc_qk = idesc_f32acc(0, 0, 128, 64, 0, 0);     // fp16 x fp16, K-major
+      // Q.C^T in the source's type (bf16 Q in TMEM for a bf16 cache), P.V in fp16
+      constexpr uint32_t kQkFmt = FP16_SRC ? 0u : kFmtBF16;
+      constexpr uint32_t idesc_qk = idesc_f32acc(kQkFmt, kQkFmt, 128, 64, 0, 0);   // K-major
       constexpr uint32_t idesc_pv = idesc_f32acc(0, 0, 128, 256, 0, 1);    // P K-major, V MN-major
       bool ok = mbar_wait(&bar->q_full, 0, p.budget);
       if (!ok) report_error(p.err, kDevErrTimeout, 320, 0);
@@ -421,6 +446,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                         smem_desc(kv_addr + KV_ROPE + k * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
           }
           umma_commit(&bar->s_full);
+          if constexpr (!FP16_SRC) umma_commit(&bar->qk_done[st]);
         }
         if (i >= 2) {
           const int j = i - 2;
@@ -428,8 +454,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
             report_error(p.err, kDevErrTimeout, 322, j);
             break;
           }
-          tc_fence_after();
           const int st = j % kStages;
+          if (!FP16_SRC && !mbar_wait(&bar->v_full[st], (j / kStages) & 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 323, j);
+            break;
+          }
+          tc_fence_after();
           const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -534,7 +564,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                                     : 4 * kQBox + h * 64 + (((u - 32) ^ ((h >> 1) & 3)) << 4);
         uint4 raw = make_uint4(0, 0, 0, 0);
         if (ok && h < H) raw = *reinterpret_cast<const uint4*>(sQ + off);
-        const uint4 v = cvt_unit(raw);
+        const uint4 v = FP16_SRC ? cvt_unit(raw) : raw;   // Q in the type of the gathered entries
         qv[4 * m + 0] = v.x;
         qv[4 * m + 1] = v.y;
         qv[4 * m + 2] = v.z;
