@@ -81,6 +81,23 @@ def work_model(x):
             "sparse_mla": {"flops": mla_flops, "bytes": mla_bytes, "peak": "bf16"}}
 
 
+def prep_work(total_q):
+    """Bytes of the upstream preparation of one batch: the FP8 quantiser over q
+    (total_q x 64 vectors: 256 B read, 128 + 4 B written each) and the cache
+    write of the new tokens (key 256 B read, 132 B written; latent 1152 B read
+    and written)."""
+    return {"quantize_q": {"flops": 0, "bytes": total_q * 64 * (256 + 128 + 4), "peak": None},
+            "cache_write": {"flops": 0, "bytes": total_q * (256 + 132 + 2 * 1152), "peak": None}}
+
+
+def prep_line(prep_sec, total_q, pk):
+    """The preparation kernels' times against their HBM roofline (not part of `value`)."""
+    if prep_sec is None or "error" in prep_sec:
+        return prep_sec
+    w = prep_work(total_q)
+    return {n: roofline_entry(n, w[n], prep_sec[n], pk) for n in w}
+
+
 def roofline_entry(stage, work, sec, pk, sustained=True):
     tf = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
     tensor_peak = {"fp8": 2.0 * tf, "bf16": tf, None: None}[work["peak"]]
@@ -442,6 +459,36 @@ def main():
     e2e_sec = slowest_rank(e_start.elapsed_time(e_end) / 1e3, pg, dev)
     e2e_value = whole_job_rate(world, b.total_q, args.steps, e2e_sec)
 
+    # ---- upstream preparation, outside the step: the per-128 FP8 quantiser
+    # over this batch's q (bf16 -> codes + scales) and the write of its new
+    # tokens' keys and latent rows into caches of the workload's size ----
+    prep_sec = None
+    try:
+        gen = torch.Generator(device=dev).manual_seed(1234 + rank)
+        q_bf = torch.randn((b.total_q, 64, 128), generator=gen, device=dev).to(torch.bfloat16)
+        k_bf = torch.randn((b.total_q, 128), generator=gen, device=dev).to(torch.bfloat16)
+        lat_bf = torch.randn((b.total_q, 576), generator=gen, device=dev).to(torch.bfloat16)
+        q8p = torch.empty((b.total_q, 64, 128), dtype=torch.uint8, device=dev)
+        qsp = torch.empty((b.total_q, 64), dtype=torch.float32, device=dev)
+        k8c, ksc, latc = torch.empty_like(t["k8"]), torch.empty_like(t["k_scale"]), torch.empty_like(t["latent"])
+        ws_p = dsa.workspace(dsa.OP_CACHE_WRITE, batch, 0, 0, device=dev)
+        pe = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            flush.fill_(float(i))
+            e = pe[i - args.warmup] if i >= args.warmup else None
+            if e: e[0].record(stream)
+            dsa.quantize_fp8(q_bf, q8p, qsp)
+            if e: e[1].record(stream)
+            dsa.cache_write(batch, k_bf, lat_bf, k8c, ksc, latc, ws_p)
+            if e: e[2].record(stream)
+        torch.cuda.synchronize()
+        dsa.check_device_error(ws_p)
+        prep_sec = {"quantize_q": sum(e[0].elapsed_time(e[1]) for e in pe) / 1e3 / args.steps,
+                    "cache_write": sum(e[1].elapsed_time(e[2]) for e in pe) / 1e3 / args.steps}
+        del q_bf, k_bf, lat_bf, q8p, qsp, k8c, ksc, latc
+    except Exception as exc:     # reported in the line; the step's numbers above stand
+        prep_sec = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+
     if pg:
         pg.barrier()
         pg.destroy_process_group()
@@ -470,7 +517,8 @@ def main():
             "stages": {n: {k2: v for k2, v in s.items()} for n, s in stages.items()},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
+            "prep": prep_line(prep_sec, b.total_q, pk)}
     print(json.dumps(line), flush=True)
     return 0
 

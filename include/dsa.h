@@ -23,6 +23,8 @@
  *   dsa_forward         indexer -> top-k -> sparse MLA on one stream
  *                       (T_DSA = T_index + T_topk + T_gather + T_sparse_attn,
  *                       "DeepSeek V3.2 稀疏注意力", complexity section).
+ *   dsa_quantize_fp8,   upstream of the three: the per-128 FP8 quantiser of q / k
+ *   dsa_cache_write     and the write of new tokens into the key and latent caches.
  *
  * Conventions (all entry points):
  *   - Every tensor pointer is caller-owned DEVICE memory, row-major and
@@ -77,7 +79,8 @@ typedef enum {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA = 2,
-  DSA_OP_FORWARD = 3
+  DSA_OP_FORWARD = 3,
+  DSA_OP_CACHE_WRITE = 4
 } dsa_op_t;
 
 /* Host struct describing a ragged batch; the three arrays are DEVICE memory. */
@@ -182,6 +185,39 @@ DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, co
 DSA_API dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* batch, const void* q, int32_t n_heads,
                                              const void* kv, const int32_t* idx, int32_t k_sel, float sm_scale,
                                              void* out, float* lse, dsa_stream_t stream);
+
+/* Upstream preparation ("详解DSA", the indexer code: q and k pass through a
+ * per-block activation quantiser with block = the indexer head dim, one fp32
+ * scale per 128-element vector, and the new tokens' codes and scales are
+ * stored in the key cache; "DeepSeek V3.2 稀疏注意力", data-flow section: the
+ * latent rows go to the MLA cache).  Scale rule (open on the page; the plain
+ * reading): scale = fp32(amax / 448) over the vector's values, 1 for an
+ * all-zero vector; code = e4m3(fp32(x / scale)), round to nearest even,
+ * saturating at +-448, sign of zero kept.  Inputs must be finite.
+ *
+ * dsa_quantize_fp8: n_vec vectors of 128 bf16 values.
+ *   x      [n_vec, 128] bf16
+ *   codes  [n_vec, 128] e4m3 out
+ *   scales [n_vec] fp32 out
+ *   n_vec >= 0 (0: nothing launched); e.g. q as [total_q * 64, 128] gives the
+ *   q_fp8 / q_scale inputs of dsa_indexer_scores.  No workspace, no device
+ *   error word (there is no index to check). */
+DSA_API dsa_status_t dsa_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales,
+                                      dsa_stream_t stream);
+
+/* dsa_cache_write: the keys and latent rows of the batch's new tokens into the
+ * flat caches.  Query row r (sequence b, position t, see "Ragged batches")
+ * writes cache row kv_start[b] + t:
+ *   k       [total_q, 128] bf16 new keys     -> k_cache [total_keys, 128] e4m3,
+ *                                               k_scale [total_keys] fp32 (the rule above)
+ *   latent  [total_q, 576] bf16 new entries  -> latent_cache [total_keys, 576] bf16 (copied)
+ * Other cache rows are untouched.  ws: at least dsa_workspace_size(
+ * DSA_OP_CACHE_WRITE, ...) bytes; a sequence whose cu_q / kv_len / kv_start
+ * would address rows outside the caches is skipped and DSA_ERR_DEVICE_BOUNDS
+ * recorded in the device error word. */
+DSA_API dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* k, const void* latent, void* k_cache,
+                                     float* k_scale, void* latent_cache, void* ws, size_t ws_bytes,
+                                     dsa_stream_t stream);
 
 /* Synchronise `stream`, read the device error word of `ws`, clear it, and
  * return DSA_OK, DSA_ERR_DEVICE_TIMEOUT or DSA_ERR_DEVICE_BOUNDS (or

@@ -22,7 +22,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdsa.so")
 
-OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_CACHE_WRITE = 0, 1, 2, 3, 4
 INDEX_HEADS, INDEX_DIM, LATENT_DIM, VALUE_DIM, MAX_K_SEL = 64, 128, 576, 512, 2048
 
 STATUS = {
@@ -47,6 +47,8 @@ EXPORTS = [
     "dsa_status_string",
     "dsa_version",
     "dsa_forward_launches",
+    "dsa_quantize_fp8",
+    "dsa_cache_write",
 ]
 
 
@@ -102,6 +104,10 @@ def _lib():
         lib.dsa_version.restype = I32
         lib.dsa_forward_launches.argtypes = [BP, I32, I32]
         lib.dsa_forward_launches.restype = I32
+        lib.dsa_quantize_fp8.argtypes = [P, I64, P, P, P]
+        lib.dsa_quantize_fp8.restype = ctypes.c_int
+        lib.dsa_cache_write.argtypes = [BP, P, P, P, P, P, P, SZ, P]
+        lib.dsa_cache_write.restype = ctypes.c_int
         _LIB = lib
     return _LIB
 
@@ -205,6 +211,18 @@ def forward(batch: Batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel: int, q, kv, 
     _check(_lib().dsa_forward(batch.ref, _ptr(q_fp8), _ptr(q_scale), _ptr(w), _ptr(k_fp8), _ptr(k_scale), k_sel,
                               _ptr(q), n_heads, _ptr(kv), float(sm_scale), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
                               ws.numel(), _stream(stream)), "dsa_forward")
+
+
+def quantize_fp8(x, codes, scales, stream=None):
+    """Per-128 FP8 e4m3 quantisation: x bf16 [..., 128] -> codes uint8 [..., 128], scales fp32 [...]."""
+    n_vec = x.numel() // INDEX_DIM
+    _check(_lib().dsa_quantize_fp8(_ptr(x), n_vec, _ptr(codes), _ptr(scales), _stream(stream)), "dsa_quantize_fp8")
+
+
+def cache_write(batch: Batch, k, latent, k_cache, k_scale, latent_cache, ws, stream=None):
+    """New tokens' keys (FP8 + scale) and latent rows into the flat caches at their positions."""
+    _check(_lib().dsa_cache_write(batch.ref, _ptr(k), _ptr(latent), _ptr(k_cache), _ptr(k_scale), _ptr(latent_cache),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "dsa_cache_write")
 
 
 def check_device_error(ws, stream=None):

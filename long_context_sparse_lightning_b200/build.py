@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdsa.so")
-SOURCES = ["api.cu", "api_no_alloc.cu", "indexer_sm100.cu", "topk.cu", "sparse_mla_sm100.cu"]
+SOURCES = ["api.cu", "api_no_alloc.cu", "indexer_sm100.cu", "topk.cu", "sparse_mla_sm100.cu", "prep.cu"]
 HEADERS = ["ptx.cuh", "kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -279,6 +279,8 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, 
     case DSA_OP_SPARSE_MLA:
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
       return kHeaderBytes + mla_ws_bytes(batch, k_sel);
+    case DSA_OP_CACHE_WRITE:
+      return kHeaderBytes;
     case DSA_OP_FORWARD: {
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
       const size_t scores = align_up(static_cast<size_t>(batch->total_q) * forward_ld(batch) * sizeof(float), 256);
@@ -363,6 +365,34 @@ int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, int32_t n_
   n += 1;                                                                    // sparse MLA
   if (mla_split(batch, k_sel).nsplit > 1) n += 1;                            // merge
   return n;
+}
+
+dsa_status_t dsa_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales, dsa_stream_t stream) {
+  if (n_vec < 0 || x == nullptr || codes == nullptr || scales == nullptr) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return DSA_ERR_INVALID_ARG;
+  if (n_vec >= (int64_t(1) << 40)) return DSA_ERR_UNSUPPORTED;
+  if (n_vec == 0) return DSA_OK;
+  return dsa::launch_quantize_fp8(x, n_vec, codes, scales, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DSA_OK
+             : DSA_ERR_CUDA;
+}
+
+dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* k, const void* latent, void* k_cache,
+                             float* k_scale, void* latent_cache, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if (k == nullptr || latent == nullptr || k_cache == nullptr || k_scale == nullptr || latent_cache == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(latent) || !aligned16(k_cache) || !aligned16(k_scale) || !aligned16(latent_cache))
+    return DSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  return dsa::launch_cache_write(batch->num_seqs, batch->max_q_per_seq, batch->total_q, batch->total_keys,
+                                 batch->cu_q, batch->kv_len, batch->kv_start, k, latent, k_cache, k_scale,
+                                 latent_cache, static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? DSA_OK
+             : DSA_ERR_CUDA;
 }
 
 dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info) {

@@ -110,4 +110,13 @@ cudaError_t launch_sparse_mla_fp16(dim3 grid, const MlaParams& p, const MlaMaps&
 cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream);
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream);
 
+// ------------------------------------------------------------------- prep --
+// per-128 FP8 quantiser: x bf16 [n_vec, 128] -> codes e4m3 [n_vec, 128], scales [n_vec]
+cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales, cudaStream_t stream);
+// new tokens' keys (quantised) and latent rows into the flat caches
+cudaError_t launch_cache_write(int num_seqs, int max_q_per_seq, int total_q, int64_t total_keys,
+                               const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start, const void* k,
+                               const void* latent, void* k_cache, float* k_scale, void* latent_cache, uint32_t* err,
+                               cudaStream_t stream);
+
 }  // namespace dsa

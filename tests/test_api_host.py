@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     txt = open(os.path.join(ROOT, "include", "dsa.h")).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", txt)))
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", txt)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -121,3 +121,23 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(dsa, "_LIB", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         dsa.library()
+
+
+def test_prep_entry_points_reject_bad_arguments():
+    lib = dsa.library()
+    c = _host_batch()
+    ref = ctypes.byref(c)
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    # quantiser: negative count, null or misaligned pointers; an empty call is a no-op
+    assert lib.dsa_quantize_fp8(fake, -1, fake, fake, None) == 1
+    assert lib.dsa_quantize_fp8(None, 4, fake, fake, None) == 1
+    assert lib.dsa_quantize_fp8(fake, 4, P(0x10004), fake, None) == 1
+    assert lib.dsa_quantize_fp8(fake, 0, fake, fake, None) == 0
+    # cache write: workspace size, null / misaligned caches, empty batch
+    assert lib.dsa_workspace_size(dsa.OP_CACHE_WRITE, ref, 0, 0) == 256
+    assert lib.dsa_cache_write(ref, fake, fake, fake, fake, None, fake, 256, None) == 1
+    assert lib.dsa_cache_write(ref, fake, P(0x10008), fake, fake, fake, fake, 256, None) == 1
+    assert lib.dsa_cache_write(ref, fake, fake, fake, fake, fake, fake, 16, None) == 4
+    empty = _host_batch(total_q=0, max_q=0)
+    assert lib.dsa_cache_write(ctypes.byref(empty), fake, fake, fake, fake, fake, fake, 256, None) == 0
