@@ -8,6 +8,9 @@
 
 namespace dsa {
 
+// SMs of the current device (queried once per device)
+int sm_count();
+
 // ---------------------------------------------------------------- indexer --
 struct IndexerParams {
   const int32_t* cu_q;

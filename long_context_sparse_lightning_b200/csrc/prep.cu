@@ -108,10 +108,8 @@ __global__ void __launch_bounds__(kWarps * 32) cache_write_kernel(const CacheWri
 }  // namespace
 
 cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales, cudaStream_t stream) {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t need = (n_vec + kWarps * kUnroll - 1) / (kWarps * kUnroll);
-  const int64_t cap = static_cast<int64_t>(sms) * 8;     // 8 CTAs (64 warps) per SM, then grid-stride
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;     // 8 CTAs (64 warps) per SM, then grid-stride
   const int grid = static_cast<int>(need < cap ? need : cap);
   quantize_fp8_kernel<<<grid, kWarps * 32, 0, stream>>>(static_cast<const uint2*>(x), n_vec,
                                                         static_cast<uint32_t*>(codes), scales);

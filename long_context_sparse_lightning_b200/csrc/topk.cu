@@ -806,18 +806,6 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p
   for (int j = tid; j < k; j += BLOCK) out[j] = __ldcg(&cpos[__ldcg(&out[j])]);   // candidate -> position
 }
 
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    cached[dev] = v;
-  }
-  return cached[dev];
-}
-
 template <int BLOCK, int EPT, int MIN_CTAS>
 cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
   constexpr size_t smem = reg_smem_bytes<BLOCK, EPT>();
@@ -830,6 +818,18 @@ cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int sm_count() {
+  static int cached[64] = {0};   // written once per device with the same value: a benign race
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
 
 TopkSegments topk_segments(int max_kv_len, int k_sel, int total_q) {
   TopkSegments t{0, 0};
