@@ -25,6 +25,7 @@
 // engine streams its next row into shared memory.  Longer rows run one CTA
 // per row and re-read the row from global memory (L2) on every pass.
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 
 #include "kernels.cuh"
@@ -820,15 +821,16 @@ cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
 }  // namespace
 
 int sm_count() {
-  static int cached[64] = {0};   // written once per device with the same value: a benign race
+  // per-device cache; concurrent first calls store the same value
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int v = 0;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    cached[dev] = v;
+    cached[dev].store(v, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return v;
 }
 
 TopkSegments topk_segments(int max_kv_len, int k_sel, int total_q) {
