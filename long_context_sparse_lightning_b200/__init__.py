@@ -215,6 +215,9 @@ def forward(batch: Batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel: int, q, kv, 
 
 def quantize_fp8(x, codes, scales, stream=None):
     """Per-128 FP8 e4m3 quantisation: x bf16 [..., 128] -> codes uint8 [..., 128], scales fp32 [...]."""
+    if x.dtype != torch.bfloat16 or x.shape[-1] != INDEX_DIM or codes.dtype != torch.uint8 \
+            or codes.numel() != x.numel() or scales.dtype != torch.float32 or scales.numel() * INDEX_DIM != x.numel():
+        raise ValueError("quantize_fp8: x bf16 [..., 128], codes uint8 of the same size, scales fp32 [...]")
     n_vec = x.numel() // INDEX_DIM
     _check(_lib().dsa_quantize_fp8(_ptr(x), n_vec, _ptr(codes), _ptr(scales), _stream(stream)), "dsa_quantize_fp8")
 

@@ -141,3 +141,14 @@ def test_prep_entry_points_reject_bad_arguments():
     assert lib.dsa_cache_write(ref, fake, fake, fake, fake, fake, fake, 16, None) == 4
     empty = _host_batch(total_q=0, max_q=0)
     assert lib.dsa_cache_write(ctypes.byref(empty), fake, fake, fake, fake, fake, fake, 256, None) == 0
+
+
+def test_quantize_binding_checks_shapes_before_the_call():
+    x = torch.zeros((3, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dsa.quantize_fp8(x, torch.zeros((3, 128), dtype=torch.uint8), torch.zeros(2, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        dsa.quantize_fp8(x.float(), torch.zeros((3, 128), dtype=torch.uint8), torch.zeros(3, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        dsa.quantize_fp8(torch.zeros((3, 64), dtype=torch.bfloat16), torch.zeros((3, 64), dtype=torch.uint8),
+                         torch.zeros(3, dtype=torch.float32))
