@@ -18,6 +18,10 @@ idx, lse) back; consecutive steps overlap on three streams (copy in, compute,
 copy out) over double-buffered device buffers, as a serving loop runs them, and
 the timed region spans the first copy in to the last copy out.
 
+The prep object times the upstream preparation of the same batch outside the
+step (the per-128 FP8 quantiser over its q, the cache write of its new
+tokens) against the HBM roofline; it is not part of `value`.
+
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (rank 0 only).
 """
