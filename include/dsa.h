@@ -137,9 +137,13 @@ DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int
  *   lse  [total_q, n_heads] fp32 natural-log sum-exp of the scaled logits, or NULL.
  *   A row with no usable entry gives out = 0, lse = -inf.
  *   1 <= n_heads <= 128 (one 128-row MMA tile; fewer heads leave rows idle);
- *   k_sel as for dsa_topk.  Internally q and the gathered entries are
- *   converted to fp16 (exact for |x| in [2^-14, 65504]; larger magnitudes
- *   saturate) and the softmax probabilities are rounded to fp16. */
+ *   k_sel as for dsa_topk.  Internally the value part of the gathered entries
+ *   is converted to fp16 (exact for |x| in [2^-14, 65504]; larger magnitudes
+ *   saturate) and the softmax probabilities are rounded to fp16.  The scores
+ *   q . c use the bf16 values as given, except for batches whose selections
+ *   reuse each cache row many times (prefill-shaped), where the library first
+ *   makes an fp16 copy of the cache in `ws` and q and the whole entries go
+ *   through the same fp16 conversion. */
 DSA_API dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
                             const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
                             size_t ws_bytes, dsa_stream_t stream);
