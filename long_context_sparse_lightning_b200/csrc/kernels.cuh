@@ -104,8 +104,9 @@ struct MlaMaps {
 // Encodes the three descriptors for q [total_q * n_heads, 576] and out
 // [total_q * n_heads, 512]; false if the driver refuses them.
 bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads);
-// p.kv is the bf16 cache: selected rows are gathered with 16-byte loads and
-// converted to fp16 in shared memory (no extra buffers).
+// p.kv is the bf16 cache: selected rows are gathered with 16-byte loads, Q.C^T
+// runs in bf16 on them, and their value part is then converted to fp16 in
+// shared memory for P.V (no extra buffers).
 cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
 // p.kv is an fp16 copy of the cache (launch_latent_to_fp16): rows are
 // gathered ready for the MMAs.
