@@ -22,6 +22,16 @@ The prep object times the upstream preparation of the same batch outside the
 step (the per-128 FP8 quantiser over its q, the cache write of its new
 tokens) against the HBM roofline; it is not part of `value`.
 
+On one GPU the line also carries `workloads`: the forward step and its three
+stages, each against its roofline, for the other four configurations (decode
+at 16K-32K context, speculative decode at 128K, the 8K prefill and the tiny
+prefill), so one run reports all five.  `--no-extra-workloads` skips them.
+
+Roofline denominators: MEASURED_PEAKS.json's HBM copy bandwidth and burst
+bf16 GEMM rate (each stage is timed on its own, not inside a seconds-long
+loop), and an FP8 e4m3 GEMM rate measured at the start of the run
+(torch._scaled_mm), 2 x bf16 if that probe fails.
+
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (rank 0 only).
 """
@@ -51,13 +61,47 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def peaks():
+    """Roofline denominators: MEASURED_PEAKS.json (HBM copy bandwidth and the
+    burst cuBLAS bf16 GEMM rate) when present, else the profiling fallback.
+    Each stage is timed on its own (per-launch CUDA events over a short loop),
+    so the burst GEMM figure is the matching denominator, not the sustained one.
+    The FP8 peak is filled in by fp8_peak_probe() at run time."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             m = json.load(f)
-        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
-                "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+        pk = {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"], "source": "measured"}
+    else:
+        pk = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+    pk["fp8_tflops"] = 2.0 * pk["bf16_tflops"]
+    pk["fp8_source"] = "2 x bf16 burst (nominal dense FP8/bf16 ratio)"
+    return pk
+
+
+def fp8_peak_probe(dev, n=8192, reps=10):
+    """Burst FP8 e4m3 dense GEMM rate (torch._scaled_mm, n^3, best of `reps`,
+    CUDA events): the denominator of the FP8 indexer's tensor roofline.
+    Returns (TFLOP/s, description) or (None, reason)."""
+    import torch
+    try:
+        g = torch.Generator(device=dev).manual_seed(99)
+        a = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), generator=g, device=dev).to(torch.float8_e4m3fn).t()   # column-major operand
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1) / 1e3)
+        del a, b
+        return 2.0 * n ** 3 / best / 1e12, f"measured: torch._scaled_mm e4m3 {n}^3, best of {reps} (burst)"
+    except Exception as exc:   # the nominal ratio stands in
+        return None, f"probe failed ({type(exc).__name__}); 2 x bf16 burst"
 
 
 # ----------------------------------------------------------------- work model
@@ -102,18 +146,21 @@ def prep_line(prep_sec, total_q, pk):
     return {n: roofline_entry(n, w[n], prep_sec[n], pk) for n in w}
 
 
-def roofline_entry(stage, work, sec, pk, sustained=True):
-    tf = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    tensor_peak = {"fp8": 2.0 * tf, "bf16": tf, None: None}[work["peak"]]
+def roofline_entry(stage, work, sec, pk):
+    """One stage against its roofline: the slower of its FLOPs at the tensor
+    peak of its type (burst) and its algorithmic bytes at the HBM peak decides
+    the bound; achieved = that work / the measured time."""
+    tensor_peak = {"fp8": pk["fp8_tflops"], "bf16": pk["bf16_tflops"], None: None}[work["peak"]]
     t_flops = work["flops"] / (tensor_peak * 1e12) if tensor_peak else 0.0
     t_bytes = work["bytes"] / (pk["hbm_gbs"] * 1e9)
     if t_flops >= t_bytes:
         achieved = work["flops"] / sec / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": achieved / tensor_peak, "ideal_us": t_flops * 1e6, "us": sec * 1e6}
+                "frac": achieved / tensor_peak, "ideal_us": t_flops * 1e6, "us": sec * 1e6,
+                "work": work["flops"]}
     achieved = work["bytes"] / sec / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / pk["hbm_gbs"], "ideal_us": t_bytes * 1e6, "us": sec * 1e6}
+            "frac": achieved / pk["hbm_gbs"], "ideal_us": t_bytes * 1e6, "us": sec * 1e6, "work": work["bytes"]}
 
 
 def ncu_traffic(kernel_file, kernel_key):
@@ -312,39 +359,19 @@ def config_of(x, args):
             "l2": "flushed between timed steps (256 MiB write, outside the events)", "seed": 0}
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference step")
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    args.warmup = max(3, args.warmup)
-    world, rank, local = dist_setup(args)
-    if args.impl == "reference":
-        return run_reference(args, world, rank)
+EXTRA_WORKLOADS = ["decode_64x16k_32k", "spec_decode_8x2_128k", "prefill_8k", "tiny_prefill_512"]
 
+
+def measure(x, args, dev, pg, world, full, min_region_s=0.0):
+    """Time the forward step of one workload on resident inputs (L2 flushed
+    between steps), then each stage on its own; with `full`, also end to end
+    from pinned host buffers and the upstream preparation kernels."""
     import torch
     import long_context_sparse_lightning_b200 as dsa
-    from dsa_inputs import make_inputs
     from dsa_inputs.torch_io import host_tensors
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as td
-        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = td
-
-    x = make_inputs(args.workload, seed=rank)
     b = x.batch
-    host = host_tensors(x, pin=True)
+    host = host_tensors(x, pin=full)
     t = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
     batch = dsa.Batch(t["cu_q"], t["kv_len"], t["kv_start"], b.total_q, b.max_q_per_seq, b.max_kv_len, b.total_keys)
     k, H = x.k_sel, x.n_heads
@@ -360,17 +387,25 @@ def main():
         dsa.forward(batch, t["q8"], t["q_scale"], t["w"], t["k8"], t["k_scale"], k, t["q_mla"], t["latent"],
                     x.sm_scale, idx, out, lse, ws)
 
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for _ in range(args.warmup):
         step()
+    w1.record(stream)
+    torch.cuda.synchronize()
     dsa.check_device_error(ws)
+    steps = args.steps
+    if min_region_s > 0:        # short steps: enough of them for the clock samples to mean something
+        per = w0.elapsed_time(w1) / 1e3 / args.warmup
+        steps = int(min(500, max(steps, math.ceil(min_region_s / max(per, 1e-6)))))
 
-    # ---- headline: K steps on resident inputs, L2 flushed between steps ----
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # ---- K steps on resident inputs, L2 flushed between steps ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
+    with ClockSampler(dev.index) as clk:
+        for i in range(steps):
             flush.fill_(float(i))
             ev[i][0].record(stream)
             step()
@@ -380,8 +415,8 @@ def main():
         pg.barrier()
     dsa.check_device_error(ws)
     sec = slowest_rank(sum(a.elapsed_time(c) for a, c in ev) / 1e3, pg, dev)
-    value = whole_job_rate(world, b.total_q, args.steps, sec)
-    launches_per_step = dsa.forward_launches(batch, k, H)
+    res = {"steps": steps, "sec": sec, "value": whole_job_rate(world, b.total_q, steps, sec),
+           "launches_per_step": dsa.forward_launches(batch, k, H), "clocks": clk.summary()}
 
     # ---- per-stage device time (same stream, CUDA events between the launches) ----
     ld = ((b.max_kv_len + 3) // 4) * 4
@@ -389,8 +424,8 @@ def main():
     # one workspace for the three standalone stages: the largest of their sizes
     ws_op = max((dsa.OP_TOPK, dsa.OP_SPARSE_MLA), key=lambda op: dsa.workspace_size(op, batch, k, H))
     ws_s = dsa.workspace(ws_op, batch, k, H, device=dev)
-    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for i in range(args.warmup + args.steps):
+    st_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(args.warmup + steps):
         flush.fill_(float(i))
         e = st_ev[i - args.warmup] if i >= args.warmup else None
         if e: e[0].record(stream)
@@ -402,9 +437,11 @@ def main():
         if e: e[3].record(stream)
     torch.cuda.synchronize()
     dsa.check_device_error(ws_s)
-    stage_sec = {name: sum(e[j].elapsed_time(e[j + 1]) for e in st_ev) / 1e3 / args.steps
-                 for j, name in enumerate(["indexer", "topk", "sparse_mla"])}
-    del scores
+    res["stage_sec"] = {name: sum(e[j].elapsed_time(e[j + 1]) for e in st_ev) / 1e3 / steps
+                        for j, name in enumerate(["indexer", "topk", "sparse_mla"])}
+    del scores, ws_s
+    if not full:
+        return res
 
     # ---- end to end through the C ABI from pinned host buffers ----
     # Every step copies all of its inputs in and its results (out, idx, lse)
@@ -454,21 +491,23 @@ def main():
     torch.cuda.synchronize()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(s_in)
-    for i in range(args.warmup, args.warmup + args.steps):
+    for i in range(args.warmup, args.warmup + steps):
         e2e_step(i)
     e_end.record(s_out)
     torch.cuda.synchronize()
     for _, _, _, wsj in sets:
         dsa.check_device_error(wsj)
     e2e_sec = slowest_rank(e_start.elapsed_time(e_end) / 1e3, pg, dev)
-    e2e_value = whole_job_rate(world, b.total_q, args.steps, e2e_sec)
+    res["e2e"] = {"value": whole_job_rate(world, b.total_q, steps, e2e_sec), "unit": UNIT,
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del sets, t2
 
     # ---- upstream preparation, outside the step: the per-128 FP8 quantiser
     # over this batch's q (bf16 -> codes + scales) and the write of its new
     # tokens' keys and latent rows into caches of the workload's size ----
     prep_sec = None
     try:
-        gen = torch.Generator(device=dev).manual_seed(1234 + rank)
+        gen = torch.Generator(device=dev).manual_seed(1234 + dev.index)
         q_bf = torch.randn((b.total_q, 64, 128), generator=gen, device=dev).to(torch.bfloat16)
         k_bf = torch.randn((b.total_q, 128), generator=gen, device=dev).to(torch.bfloat16)
         lat_bf = torch.randn((b.total_q, 576), generator=gen, device=dev).to(torch.bfloat16)
@@ -476,8 +515,8 @@ def main():
         qsp = torch.empty((b.total_q, 64), dtype=torch.float32, device=dev)
         k8c, ksc, latc = torch.empty_like(t["k8"]), torch.empty_like(t["k_scale"]), torch.empty_like(t["latent"])
         ws_p = dsa.workspace(dsa.OP_CACHE_WRITE, batch, 0, 0, device=dev)
-        pe = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        for i in range(args.warmup + args.steps):
+        pe = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(args.warmup + steps):
             flush.fill_(float(i))
             e = pe[i - args.warmup] if i >= args.warmup else None
             if e: e[0].record(stream)
@@ -487,11 +526,67 @@ def main():
             if e: e[2].record(stream)
         torch.cuda.synchronize()
         dsa.check_device_error(ws_p)
-        prep_sec = {"quantize_q": sum(e[0].elapsed_time(e[1]) for e in pe) / 1e3 / args.steps,
-                    "cache_write": sum(e[1].elapsed_time(e[2]) for e in pe) / 1e3 / args.steps}
+        prep_sec = {"quantize_q": sum(e[0].elapsed_time(e[1]) for e in pe) / 1e3 / steps,
+                    "cache_write": sum(e[1].elapsed_time(e[2]) for e in pe) / 1e3 / steps}
         del q_bf, k_bf, lat_bf, q8p, qsp, k8c, ksc, latc
     except Exception as exc:     # reported in the line; the step's numbers above stand
         prep_sec = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+    res["prep_sec"] = prep_sec
+    return res
+
+
+def stage_lines(x, stage_sec, pk):
+    wm = work_model(x)
+    return {n: roofline_entry(n, wm[n], stage_sec[n], pk) for n in stage_sec}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference step")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="measure only --workload (by default a 1-GPU run also measures the other four configs)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    from dsa_inputs import make_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = td
+
+    x = make_inputs(args.workload, seed=rank)
+    r = measure(x, args, dev, pg, world, full=True)
+    extra = {}
+    if world == 1 and not args.no_extra_workloads:
+        for name in EXTRA_WORKLOADS:
+            if name == args.workload:
+                continue
+            xe = make_inputs(name, seed=rank)
+            re_ = measure(xe, args, dev, None, world, full=False, min_region_s=0.05)
+            extra[name] = (xe, re_)
+            torch.cuda.empty_cache()
+    pk = peaks()
+    fp8, fp8_src = fp8_peak_probe(dev)
+    if fp8 is not None:
+        pk["fp8_tflops"], pk["fp8_source"] = fp8, fp8_src
+    else:
+        pk["fp8_source"] = fp8_src
 
     if pg:
         pg.barrier()
@@ -499,30 +594,36 @@ def main():
     if rank != 0:
         return 0
 
-    pk = peaks()
-    wm = work_model(x)
-    stages = {n: roofline_entry(n, wm[n], stage_sec[n], pk) for n in stage_sec}
-    dom = max(stage_sec, key=stage_sec.get)
+    stages = stage_lines(x, r["stage_sec"], pk)
+    dom = max(r["stage_sec"], key=r["stage_sec"].get)
     kfile = {"indexer": "indexer_sm100.cu", "topk": "topk.cu", "sparse_mla": "sparse_mla_sm100.cu"}[dom]
-    roof = dict(stages[dom])
+    roof = {k2: v for k2, v in stages[dom].items() if k2 != "work"}
     roof["kernel"] = dom
     roof["traffic"] = ncu_traffic(kfile, dom)
-    roof["peak_source"] = pk["source"] + (" sustained" if roof["unit"] == "TFLOP/s" else "")
+    roof["peak_source"] = pk["source"] + (" burst bf16 GEMM" if stages[dom]["peak"] == pk["bf16_tflops"] and
+                                          roof["unit"] == "TFLOP/s" else "")
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         rps, n_rows, el = oracle_rows_per_sec(x, budget_s=args.cpu_budget)
         cpu = {"value": rps, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{n_rows} query rows of {args.workload} ({el:.1f} s): fp64 scores over each row's "
                          f"causal prefix, exact top-k, sparse MLA"}
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+f16", "data": "synthetic",
+    line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * r["sec"] / r["steps"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16/f16", "data": "synthetic",
             "config": config_of(x, args), "roofline": roof,
-            "stages": {n: {k2: v for k2, v in s.items()} for n, s in stages.items()},
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
-            "prep": prep_line(prep_sec, b.total_q, pk)}
+            "stages": stages, "peaks": {k2: pk[k2] for k2 in ("hbm_gbs", "bf16_tflops", "fp8_tflops", "fp8_source",
+                                                              "source")},
+            "cpu_baseline": cpu, "e2e": r["e2e"],
+            "gpu_launches": r["launches_per_step"] * r["steps"], "clocks": r["clocks"],
+            "prep": prep_line(r["prep_sec"], x.batch.total_q, pk)}
+    if extra:
+        line["workloads"] = {
+            name: {"value": re_["value"], "unit": UNIT, "steps": re_["steps"],
+                   "ms_per_step": 1e3 * re_["sec"] / re_["steps"], "stages": stage_lines(xe, re_["stage_sec"], pk),
+                   "gpu_launches": re_["launches_per_step"] * re_["steps"], "clocks": re_["clocks"],
+                   "config": config_of(xe, args)}
+            for name, (xe, re_) in extra.items()}
     print(json.dumps(line), flush=True)
     return 0
 

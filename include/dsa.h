@@ -137,13 +137,18 @@ DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int
  *   lse  [total_q, n_heads] fp32 natural-log sum-exp of the scaled logits, or NULL.
  *   A row with no usable entry gives out = 0, lse = -inf.
  *   1 <= n_heads <= 128 (one 128-row MMA tile; fewer heads leave rows idle);
- *   k_sel as for dsa_topk.  Internally the value part of the gathered entries
- *   is converted to fp16 (exact for |x| in [2^-14, 65504]; larger magnitudes
- *   saturate) and the softmax probabilities are rounded to fp16.  The scores
- *   q . c use the bf16 values as given, except for batches whose selections
- *   reuse each cache row many times (prefill-shaped), where the library first
- *   makes an fp16 copy of the cache in `ws` and q and the whole entries go
- *   through the same fp16 conversion. */
+ *   k_sel as for dsa_topk.
+ * Arithmetic: the logits q . c accumulate in fp32 on the tensor cores and the
+ * softmax runs in fp32.  For P . V the probabilities are rounded to fp16 and
+ * the value part of the gathered entries is converted to fp16, which holds
+ * every bf16 value of magnitude 2^-17 .. 65280 exactly (smaller magnitudes
+ * keep an absolute error below 2^-25; larger ones saturate at 65504).  The
+ * logits use the bf16 values as given, except for batches whose selections
+ * reuse each cache row many times (prefill-shaped), where the library first
+ * makes an fp16 copy of the cache in `ws` and q and the whole entries go
+ * through the same fp16 conversion.  A descriptor that addresses rows outside
+ * the cache (q_len > kv_len, kv_start + kv_len > total_keys) records
+ * DSA_ERR_DEVICE_BOUNDS and leaves that sequence's rows at out = 0, lse = -inf. */
 DSA_API dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
                             const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
                             size_t ws_bytes, dsa_stream_t stream);
@@ -181,10 +186,18 @@ DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, co
  *     call's contents; each call clears the error word it needs at the start.
  *     Calls whose work overlaps on the GPU (different streams, no ordering)
  *     race on the array and must be serialised by the caller.
- *   - Device-side error statuses (bounded-wait timeouts) are recorded in the
- *     array and are not reported to the caller; use dsa_sparse_mla with a
- *     workspace and dsa_check_device_error when they are needed.
- * Arguments and results are otherwise those of dsa_sparse_mla. */
+ *   - Device-side error statuses (bounded-wait timeouts, descriptors that
+ *     address rows outside the cache) are recorded in the array and are not
+ *     reported to the caller; use dsa_sparse_mla with a workspace and
+ *     dsa_check_device_error when they are needed.  Rows of a sequence whose
+ *     descriptors are out of range come out as out = 0, lse = -inf, never as
+ *     another call's leftovers.
+ *   - It always runs the bf16-cache kernel (bf16 Q . C^T on the gathered
+ *     rows, no fp16 copy of the cache, which would need a workspace).  On the
+ *     prefill-shaped batches where dsa_sparse_mla takes its fp16-copy path the
+ *     two entry points therefore round q . c differently; both stay within the
+ *     parity tolerances.  Arguments and results are otherwise those of
+ *     dsa_sparse_mla. */
 #define DSA_NO_ALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 DSA_API dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* batch, const void* q, int32_t n_heads,
                                              const void* kv, const int32_t* idx, int32_t k_sel, float sm_scale,

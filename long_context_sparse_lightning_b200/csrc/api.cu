@@ -16,6 +16,7 @@
 namespace {
 
 using dsa::IndexerParams;
+using dsa::wait_budget;
 using dsa::MlaParams;
 using dsa::TopkParams;
 
@@ -26,14 +27,6 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-long long wait_budget() {
-  const char* s = std::getenv("DSA_WAIT_BUDGET_CYCLES");
-  if (s != nullptr) {
-    const long long v = std::atoll(s);
-    if (v > 0) return v;
-  }
-  return kDefaultBudget;
-}
 
 // ---- cuTensorMapEncodeTiled through the runtime's driver entry point ----
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -201,6 +194,7 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   p.kv = static_cast<const uint16_t*>(kv);
   p.idx = idx;
   p.total_keys = b->total_keys;
+  p.total_q = b->total_q;
   p.k_sel = k_sel;
   p.n_heads = n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
@@ -257,6 +251,15 @@ dsa_status_t check_mla_args(const void* q, int n_heads, const void* kv, int k_se
 }  // namespace
 
 namespace dsa {
+long long wait_budget() {
+  const char* s = std::getenv("DSA_WAIT_BUDGET_CYCLES");
+  if (s != nullptr) {
+    const long long v = std::atoll(s);
+    if (v > 0) return v;
+  }
+  return kDefaultBudget;
+}
+
 bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads) {
   const uint64_t rows = static_cast<uint64_t>(total_q) * static_cast<uint64_t>(n_heads);
   const uint32_t h = static_cast<uint32_t>(n_heads);

@@ -86,7 +86,11 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   if (scratch_for_current_device(&base) != cudaSuccess) return DSA_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // The previous call's contents stay in the array; only the error word must
-  // start at zero (the partial results are fully rewritten before they are read).
+  // start at zero.  Every partial result the merge reads is written by this
+  // call first: a CTA pair that processes its split writes its partial output
+  // and log-sum-exp, and a pair whose sequence descriptors are out of range
+  // writes lse = -inf for its split, which the merge turns into out = 0,
+  // lse = -inf for that row.
   if (cudaMemsetAsync(base, 0, 16, st) != cudaSuccess) return DSA_ERR_CUDA;
 
   dsa::MlaParams p;
@@ -97,6 +101,7 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   p.kv = static_cast<const uint16_t*>(kv);
   p.idx = idx;
   p.total_keys = b->total_keys;
+  p.total_q = b->total_q;
   p.k_sel = k_sel;
   p.n_heads = n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
@@ -108,7 +113,7 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   p.part_o = nsplit > 1 ? reinterpret_cast<float*>(scratch + kHeader) : nullptr;
   p.part_lse = nsplit > 1 ? reinterpret_cast<float*>(scratch + kHeader + o_bytes) : nullptr;
   p.err = reinterpret_cast<uint32_t*>(scratch);
-  p.budget = 2000000000LL;
+  p.budget = dsa::wait_budget();
   const int64_t gx = int64_t(2) * b->max_q_per_seq * nsplit;
   if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);

@@ -11,6 +11,10 @@ namespace dsa {
 // SMs of the current device (queried once per device)
 int sm_count();
 
+// clock64 cycles one bounded device wait may take before it records
+// DSA_ERR_DEVICE_TIMEOUT: DSA_WAIT_BUDGET_CYCLES if set (> 0), else ~1 s
+long long wait_budget();
+
 // ---------------------------------------------------------------- indexer --
 struct IndexerParams {
   const int32_t* cu_q;
@@ -73,6 +77,7 @@ struct MlaParams {
   const uint16_t* kv = nullptr;       // [total_keys, 576]: bf16 cache, or its fp16 copy
   const int32_t* idx = nullptr;       // [total_q, k_sel]
   int64_t total_keys = 0;
+  int32_t total_q = 0;                // rows of q / out / lse / idx
   int32_t k_sel = 0;
   int32_t n_heads = 0;
   float scale_log2 = 0.f;             // sm_scale * log2(e)

@@ -29,16 +29,15 @@
 //              instruction and measured ~6 B/clk per SM on this pattern;
 //              16-byte cp.async from 7 warps sustains several times that.)
 //   MMA warp   S_r = Q_r . C_r^T (M=128, N=64, K=288) then O_r += P . V_r (N=256);
-//   softmax    8 warps, 16 heads x 64 columns each: each warp ships its 2 KB of
-//              partial scores (fp16) to the peer with one bulk shared-to-shared
-//              copy, one tile ahead of its own use so the transfer overlaps a
-//              whole iteration, and adds the peer's fp16 partial to its own fp32
-//              one; online softmax in log2 units with a lazily refreshed max (O
-//              rescaled in TMEM only when the max grows by more than 2^8); P
-//              stored to TMEM as fp16.  The two CTAs' scores differ by the fp16
-//              rounding of one partial; each CTA normalises its own value half
-//              with its own probabilities and row sums, so each half is an exact
-//              softmax average of its scores (the log-sum-exp comes per half).
+//   softmax    8 warps, 16 heads x 64 columns each: each warp ships its 4 KB of
+//              fp32 partial scores to the peer with one bulk shared-to-shared
+//              copy, one tile ahead of its own use so the transfer overlaps most
+//              of an iteration, and adds the peer's fp32 partial to its own
+//              (IEEE addition commutes, so both CTAs of the pair hold the same
+//              fp32 scores bit for bit and compute one softmax: the same maxima,
+//              probabilities, row sums and log-sum-exp); online softmax in log2
+//              units with a lazily refreshed max (O rescaled in TMEM only when
+//              the max grows by more than 2^8); P stored to TMEM as fp16.
 //   MMA order  Q.C^T runs two tiles ahead of P.V.
 // fp16 rather than bf16 inside the MMAs: with bf16 probabilities the rounding
 // noise costs ~1e-3 mean relative error on the bf16 output; fp16 keeps ~1e-4.
@@ -64,7 +63,7 @@ constexpr int kTileKeys = 64;
 constexpr int kStages = 4;
 constexpr int KV_STAGE = 36864;          // 64 rows x (4 x 128 B latent + 64 B RoPE)
 constexpr int KV_ROPE = 32768;
-constexpr int XBLK = 2048;               // one softmax warp's partial scores: 16 heads x 64 keys fp16
+constexpr int XBLK = 4096;               // one softmax warp's partial scores: 16 heads x 64 keys fp32
 constexpr int XBUF = 8 * XBLK;           // one tile's partial scores of all 8 softmax warps
 
 constexpr uint32_t TM_O = 0;
@@ -74,9 +73,9 @@ constexpr uint32_t TM_Q = 352;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int OFF_KV = 0;
-constexpr int OFF_STG = kStages * KV_STAGE;          // 147456: outgoing partial scores, 2 buffers
-constexpr int OFF_X = OFF_STG + 2 * XBUF;            // 180224: incoming partial scores, 2 buffers
-constexpr int OFF_IDX = OFF_X + 2 * XBUF;            // 212992: int32[2048]
+constexpr int OFF_STG = kStages * KV_STAGE;          // 147456: outgoing partial scores (one tile)
+constexpr int OFF_X = OFF_STG + XBUF;                // 180224: incoming partial scores (one tile)
+constexpr int OFF_IDX = OFF_X + XBUF;                // 212992: int32[2048]
 constexpr int OFF_VALID = OFF_IDX + 2048 * 4;        // 221184: uint32[64] validity bits
 constexpr int OFF_BAR = OFF_VALID + 64 * 4;          // 221440
 constexpr int OFF_MISC = OFF_BAR + 512;
@@ -94,7 +93,7 @@ struct Bars {
   uint64_t qk_done[kStages];   // bf16 source: Q.C^T of the stage's tile has read it (MMA commit)
   uint64_t v_full[kStages];    // bf16 source: the stage's value part converted to fp16 in place
   uint64_t s_full, s_empty;
-  uint64_t x_full[2][8], x_free[2][8];   // per buffer and softmax warp
+  uint64_t x_full[8], x_free[8];   // per softmax warp: peer's partial landed / peer has read ours
   uint64_t p_full, pv_done;
   uint64_t red;            // all softmax warps have staged the output
 };
@@ -134,17 +133,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// (x, y) + the two fp16 halves of h2 (low half to x), each added in fp32 after
-// an exact widening: one mixed-precision add per value, no separate conversion.
-__device__ __forceinline__ float2 add_f32_h2(float x, float y, uint32_t h2) {
-  float rx, ry;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "add.rn.f32.f16 %0, lo, %3;\n\tadd.rn.f32.f16 %1, hi, %4;\n\t}"
-      : "=f"(rx), "=f"(ry)
-      : "r"(h2), "f"(x), "f"(y));
-  return make_float2(rx, ry);
 }
 
 // f32x2 register pairs (low element first) and their packed fma / add
@@ -213,13 +201,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   // (a one-sided exit would leave the peer waiting in barrier.cluster).
   if (tok >= q_len) return;
   const int row = q0 + tok;
+  const int H = p.n_heads;
+  if (q0 < 0 || row >= p.total_q) {          // inconsistent cu_q: nothing of this row is written
+    if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 302, b);
+    return;
+  }
   const int kv = __ldg(&p.kv_len[b]);
   const int64_t kstart = __ldg(&p.kv_start[b]);
   if (q_len > kv || kstart < 0 || kstart + kv > p.total_keys) {
     if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 301, b);
+    // The row attends to nothing: out = 0 and lse = -inf (split partials:
+    // lse = -inf, which the merge turns into the same), so no stale partial
+    // of an earlier call is ever merged into this row.
+    const float NI = __int_as_float(0xff800000);
+    if (p.nsplit == 1) {
+      for (int u = threadIdx.x; u < H * 32; u += blockDim.x) {      // 32 16-byte units of this CTA's half
+        const int h = u >> 5, c = u & 31;
+        *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(row) * H + h) * 512 + rank * 256 + c * 8) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (rank == 0 && p.lse != nullptr)
+        for (int h = threadIdx.x; h < H; h += blockDim.x) p.lse[static_cast<int64_t>(row) * H + h] = NI;
+    } else {
+      const int64_t prow = (static_cast<int64_t>(row) * p.nsplit + split) * 128;
+      for (int h = threadIdx.x; h < 128; h += blockDim.x) p.part_lse[prow * 2 + rank * 128 + h] = NI;
+    }
     return;
   }
-  const int H = p.n_heads;
   const int e_begin = split * p.keys_per_split;
   const int e_count = max(0, min(p.k_sel, e_begin + p.keys_per_split) - e_begin);
 
@@ -262,11 +270,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
     mbar_init(&bar->s_full, 1);
     mbar_init(&bar->s_empty, 8);
-    for (int i = 0; i < 2; ++i) {
-      for (int w = 0; w < 8; ++w) {
-        mbar_init(&bar->x_full[i][w], 1);   // the receiving warp's expect_tx arrival + the peer's 2 KB copy
-        mbar_init(&bar->x_free[i][w], 1);   // the peer warp's remote arrival once it has read the block
-      }
+    for (int w = 0; w < 8; ++w) {
+      mbar_init(&bar->x_full[w], 1);   // the receiving warp's expect_tx arrival + the peer's 4 KB copy
+      mbar_init(&bar->x_free[w], 1);   // the peer warp's remote arrival once it has read the block
     }
     mbar_init(&bar->p_full, 8);
     mbar_init(&bar->pv_done, 1);
@@ -486,14 +492,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     const int hA = L + static_cast<int>(lane >> 2), hB = hA + 8;
     const int ku = 2 * static_cast<int>(lane & 3u);     // this lane's key offset inside each group of 8
     const uint32_t tbase = tmem + (static_cast<uint32_t>(L) << 16);
-    // partial-score blocks: 2 KB per warp per tile; lane l's 16-byte unit k at k*512 + l*16
+    // partial-score blocks: 4 KB per warp per tile; lane l's 16-byte unit q at q*512 + l*16
     const uint32_t stg_base = smem_u32(sm + OFF_STG) + sw * XBLK;
     const uint32_t x_base = smem_u32(sm + OFF_X) + sw * XBLK;
     const uint32_t x_base_remote = mapa_shared(x_base, peer);
-    const uint32_t x_full_remote[2] = {mapa_shared(smem_u32(&bar->x_full[0][sw]), peer),
-                                       mapa_shared(smem_u32(&bar->x_full[1][sw]), peer)};
-    const uint32_t x_free_remote[2] = {mapa_shared(smem_u32(&bar->x_free[0][sw]), peer),
-                                       mapa_shared(smem_u32(&bar->x_free[1][sw]), peer)};
+    const uint32_t x_full_remote = mapa_shared(smem_u32(&bar->x_full[sw]), peer);
+    const uint32_t x_free_remote = mapa_shared(smem_u32(&bar->x_free[sw]), peer);
     const float NEG_INF = __int_as_float(0xff800000);
     const float scale = p.scale_log2;
     float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
@@ -508,9 +512,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       if (!all && lane == 0) report_error(p.err, kDevErrTimeout, site, info);
       return all;
     };
-    // S(t) of this warp's 16 heads, kept in fp32 for this CTA and rounded to
-    // fp16 pairs for the peer: pk[2k] = head rA, keys 8k+ku, 8k+ku+1;
-    // pk[2k+1] = head rB, same keys.
+    // S(t) of this warp's 16 heads, this CTA's fp32 partial over its 288 dims:
+    // s[4k], s[4k+1] = head rA, keys 8k+ku, 8k+ku+1; s[4k+2], s[4k+3] = head rB.
     // Split in two so the TMEM load's latency overlaps other work.
     auto load_s_issue = [&](int t, uint32_t (&s)[32]) -> bool {
       if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
@@ -518,33 +521,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       tmem_ld_16x256b_x8(tbase + TM_S, s);
       return true;
     };
-    auto load_s_finish = [&](const uint32_t (&s)[32], uint32_t (&pk)[16]) {
+    auto load_s_finish = [&]() {
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->s_empty);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint32_t r;
-        asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(s[2 * c + 1])),
-            "f"(__uint_as_float(s[2 * c])));
-        pk[c] = r;
-      }
     };
-    // ship this warp's block of S(t) to the peer (one 2 KB bulk copy)
-    auto send = [&](int t, const uint32_t (&pk)[16]) -> bool {
-      const int xb = t & 1;
-      if (!wwait(&bar->x_free[xb][sw], ((t >> 1) & 1) ^ 1, true, 331, t)) return false;
-      const uint32_t stg = stg_base + xb * XBUF;
+    // ship this warp's block of S(t) to the peer: one 4 KB bulk copy of the
+    // raw fp32 values.  One buffer each way: the peer's arrival on x_free
+    // (it has read our block of tile t-1) also means that copy has finished
+    // reading our staging block.
+    auto send = [&](int t, const uint32_t (&s)[32]) -> bool {
+      if (!wwait(&bar->x_free[sw], (t & 1) ^ 1, true, 331, t)) return false;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + q * 512 + lane * 16), "r"(pk[4 * q]),
-                     "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+      for (int q = 0; q < 8; ++q) {
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg_base + q * 512 + lane * 16), "r"(s[4 * q]),
+                     "r"(s[4 * q + 1]), "r"(s[4 * q + 2]), "r"(s[4 * q + 3])
                      : "memory");
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) bulk_copy_to_peer(x_base_remote + xb * XBUF, stg, XBLK, x_full_remote[xb]);
+      if (lane == 0) bulk_copy_to_peer(x_base_remote, stg_base, XBLK, x_full_remote);
       return true;
     };
 
@@ -593,16 +590,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 
     uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
     if (n_tiles > 0) {
-      uint32_t pk0[16];
       ok = ok && load_s_issue(0, cur);
       if (ok) {
-        load_s_finish(cur, pk0);
-        ok = send(0, pk0);
+        load_s_finish();
+        ok = send(0, cur);
       }
     }
     for (int i = 0; ok && i < n_tiles; ++i) {
-      // 1. start loading the next tile's partial scores; they are packed and
-      //    shipped to the peer once this tile's scores are assembled
+      // 1. start loading the next tile's partial scores; they are shipped to
+      //    the peer once this tile's scores are assembled
       const bool more = i + 1 < n_tiles;
       uint32_t snext[32];
       if (more && !load_s_issue(i + 1, snext)) {
@@ -610,31 +606,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         break;
       }
       // 2. the peer's partial scores of tile i (this warp's own barrier)
-      const int xb = i & 1;
-      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[xb][sw], XBLK);
-      if (!wwait(&bar->x_full[xb][sw], (i >> 1) & 1, true, 332, i)) {
+      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[sw], XBLK);
+      if (!wwait(&bar->x_full[sw], i & 1, true, 332, i)) {
         ok = false;
         break;
       }
-      uint32_t xp[16];
+      uint32_t xp[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(xp[4 * q]), "=r"(xp[4 * q + 1]), "=r"(xp[4 * q + 2]), "=r"(xp[4 * q + 3])
-                     : "r"(x_base + xb * XBUF + q * 512 + lane * 16)
+                     : "r"(x_base + q * 512 + lane * 16)
                      : "memory");
       }
-      // sv[2c], sv[2c+1]: the pair of pk[c] (c even: head rA, c odd: head rB)
+      // own + peer partial in fp32 (f32x2 pairs; each lane the IEEE fp32 add):
+      // the peer computes peer + own, the same sum
       float sv[32];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float2 v = add_f32_h2(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1]), xp[c]);
+        const float2 v = unpack_f32x2(add_f32x2(pack_f32x2(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
+                                                pack_f32x2(__uint_as_float(xp[2 * c]), __uint_as_float(xp[2 * c + 1]))));
         sv[2 * c] = v.x;
         sv[2 * c + 1] = v.y;
       }
       __syncwarp();
       // the values are in registers: the peer may refill the buffer
-      if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote[xb]);
+      if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote);
       // 3. mask positions past the selection / padding: key 8k + ku + e
       const uint64_t vmask = static_cast<uint64_t>(sValid[2 * i]) | (static_cast<uint64_t>(sValid[2 * i + 1]) << 32);
       if (vmask != ~uint64_t(0)) {
@@ -680,9 +677,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       const float refB = m_runB == NEG_INF ? 0.f : m_runB;
       // next tile's partial scores: wait for the TMEM load, pack, ship
       if (more) {
-        uint32_t nxt[16];
-        load_s_finish(snext, nxt);
-        if (!send(i + 1, nxt)) {
+        load_s_finish();
+        if (!send(i + 1, snext)) {
           ok = false;
           break;
         }

@@ -107,9 +107,18 @@ def check_topk(x, idx_gpu: np.ndarray, rows, k_sel):
 
 
 def check_mla(x, out_gpu: np.ndarray, lse_gpu, idx_rows: np.ndarray, rows, max_abs=o_mla.OUT_MAX_ABS,
-              mean_rel=o_mla.OUT_MEAN_REL):
+              mean_rel=o_mla.OUT_MEAN_REL, value_scale=1.0, ulp_floor=False):
     """out_gpu [len(rows), H, 512] float (from bf16), lse_gpu [len(rows), H] or None,
-    idx_rows [len(rows), k] -- the index rows the GPU attended over."""
+    idx_rows [len(rows), k] -- the index rows the GPU attended over.
+
+    ``value_scale``: the factor the latent entries were scaled by (1 for the
+    configs' N(0,1) draws).  The output is linear in the values, so the max-abs
+    bound applies to the difference divided by it; the mean relative error is
+    scale-free.  ``ulp_floor``: an element may also differ by one bf16 step of
+    its reference value -- when a peaky softmax makes outputs as large as the
+    values themselves (|o| >= 4 value scales, where one bf16 step exceeds the
+    bound), an fp32 result and the fp64 one may round to neighbouring bf16
+    numbers."""
     ref = o_mla.sparse(x, idx_rows, rows)
     sum_abs = sum_ref = 0.0
     worst = 0.0
@@ -118,7 +127,7 @@ def check_mla(x, out_gpu: np.ndarray, lse_gpu, idx_rows: np.ndarray, rows, max_a
         rb = o_mla.bf16_output(o)
         d = np.abs(out_gpu[i].astype(np.float64) - rb)
         assert np.all(np.isfinite(out_gpu[i])), f"row {r}: non-finite output"
-        worst = max(worst, float(d.max()))
+        worst = max(worst, float(d.max()) / value_scale)
         sum_abs += float(d.sum())
         sum_ref += float(np.abs(rb).sum())
         if lse_gpu is not None:

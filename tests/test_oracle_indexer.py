@@ -97,3 +97,25 @@ def test_flop_ratio_against_page_figures():
 def test_tolerance_formula():
     B = np.array([0.0, 1.0, 1000.0])
     assert np.allclose(indexer.tolerance(B), [1e-6, 1e-3 + 1e-6, 1.0 + 1e-6])
+
+
+def test_ragged_batch_offsets_every_score_against_brute_loops():
+    # Three sequences of different lengths, one or more query rows each, in
+    # flat caches: every score of every row must come from its own sequence's
+    # key rows (kv_start offset) and cover exactly s = 0..t (t = kv_len -
+    # q_len + i).  A wrong offset, a wrong causal end or a row mapped to the
+    # wrong sequence changes values or lengths here.
+    x = make_inputs(custom_workload("pin_ragged", [9, 5, 12], [2, 5, 3], k_sel=4, n_heads=16), seed=13)
+    b = x.batch
+    assert b.kv_start.tolist() == [0, 9, 14]
+    qd = fp8.dequant(x.q8, x.q_scale)
+    kd = fp8.dequant(x.k8, x.k_scale)
+    expect_t = [7, 8, 0, 1, 2, 3, 4, 9, 10, 11]
+    got = indexer.scores(x)
+    assert [t for _, t, _, _ in got] == expect_t
+    starts = [0, 0, 9, 9, 9, 9, 9, 14, 14, 14]
+    for (r, t, I, B), k0 in zip(got, starts):
+        assert I.shape == (t + 1,) and B.shape == (t + 1,)
+        for s in range(t + 1):
+            ref = brute.index_score(qd[r].tolist(), x.w[r].tolist(), kd[k0 + s].tolist())
+            assert abs(I[s] - ref) <= 1e-12 * max(1.0, B[s]), (r, s)

@@ -113,3 +113,26 @@ def test_flop_count_and_page_figures():
     with open(os.path.join(GOLDEN, "page_figures.json")) as f:
         g = json.load(f)["fp32_score_matrix_128k_bytes"]
     assert g["context"] ** 2 * 4 == pytest.approx(g["value"], rel=1e-3)
+
+
+def test_bf16_output_rounding_matches_torch():
+    # The rounding every output comparison runs through (fp64 -> fp32 -> bf16,
+    # nearest even) against torch's own float32 -> bfloat16 cast: random
+    # values over many binades, exact ties between two bf16 neighbours (odd
+    # and even lower neighbour), values next to the largest finite bf16, bf16
+    # subnormals, signed zeros.
+    import torch
+    rng = np.random.default_rng(23)
+    parts = [rng.standard_normal(20000) * np.exp2(rng.integers(-40, 40, 20000))]
+    hi = (rng.integers(0, 1 << 16, 4000, dtype=np.uint32) << np.uint32(16))
+    hi = hi[np.isfinite(hi.view(np.float32))]
+    ties = (hi | np.uint32(0x8000)).view(np.float32)                   # halfway between neighbours
+    parts.append(ties[np.isfinite(ties)].astype(np.float64))
+    parts.append(np.array([3.3895313892515355e38, 3.38e38, -3.3895e38, 1e-40, -1e-40, 9.2e-41,
+                           1.1754942e-38, 0.0, -0.0, 1.0, -1.0, 65504.0, 6.103515625e-05]))
+    x = np.concatenate(parts)
+    x = x[np.isfinite(x.astype(np.float32))]
+    got = mla.bf16_output(x)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got, ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))

@@ -4,8 +4,9 @@ Callers such as an engine plugin restricted to the buffers its host hands it,
 or a latency-critical loop that cannot afford cudaMalloc's implicit device
 synchronisation, have no workspace to give dsa_sparse_mla.  The no-alloc entry
 point keeps the split-selection partials in a fixed library-owned device array
-instead.  These tests call it through the C ABI and check it against the
-workspace-based entry point.
+instead.  These tests call it through the C ABI, twice in a row on different
+selections, and check it against the fp64 oracle and against the
+workspace-based entry point, at the parity tolerances of the other tests.
 
 This file is named so that pytest collects it last.
 """
@@ -18,6 +19,8 @@ import torch
 
 import long_context_sparse_lightning_b200 as dsa
 from dsa_inputs import custom_workload, make_inputs
+from dsa_inputs.torch_io import device_tensors
+from tests.parity import check_mla
 
 SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -40,40 +43,105 @@ def _compare(out, lse, out_ref, lse_ref):
     assert torch.allclose(lse, lse_ref, rtol=1e-4, atol=2e-3)
 
 
-@pytest.mark.gpu
-def test_no_alloc_matches_workspace_entry_point_on_two_calls():
-    # decode-shaped batch: few tokens, so the selection is split over several
-    # CTA pairs and the partial results go through the scratch array
-    x = make_inputs(custom_workload("noalloc", [4100, 3000, 5000, 2600, 6100, 3333, 4444, 2900],
-                                    [1] * 8, k_sel=2048, n_heads=128), seed=21)
-    from dsa_inputs.torch_io import device_tensors
+def _setup(x):
     t = device_tensors(x)
     b = x.batch
     batch = dsa.Batch(t["cu_q"], t["kv_len"], t["kv_start"], b.total_q, b.max_q_per_seq, b.max_kv_len,
                       b.total_keys)
-    assert dsa.workspace_size(dsa.OP_SPARSE_MLA, batch, 2048, 128) > 256   # the split path is taken
-    rng = np.random.default_rng(5)
+    return t, batch
+
+
+def _random_selection(x, rng, n_drop):
+    b = x.batch
+    k = x.k_sel
+    idx = np.full((b.total_q, k), -1, np.int32)
+    for r in range(b.total_q):
+        t = int(b.q_pos[r])
+        n = min(k - n_drop, t + 1)
+        idx[r, :n] = rng.choice(t + 1, n, replace=False)
+    return idx
+
+
+def _two_calls(x, seed):
+    """Two calls in a row on different selections: each against the oracle and
+    against dsa_sparse_mla with a workspace."""
+    t, batch = _setup(x)
+    b = x.batch
+    H, k = x.n_heads, x.k_sel
+    rng = np.random.default_rng(seed)
+    rows = list(range(b.total_q))
     results = []
     for call in range(2):
         # a different selection per call, so stale scratch from call 1 cannot pass for call 2
-        idx = np.full((b.total_q, 2048), -1, np.int32)
-        for r in range(b.total_q):
-            kv = int(b.kv_len[r])
-            n = 2048 - 300 * call
-            idx[r, :n] = rng.choice(kv, n, replace=False)
+        idx = _random_selection(x, rng, n_drop=(k // 7) * call)
         idx_d = torch.from_numpy(idx).cuda()
-        out_ref = torch.empty((b.total_q, 128, 512), dtype=torch.bfloat16, device="cuda")
-        lse_ref = torch.empty((b.total_q, 128), dtype=torch.float32, device="cuda")
-        ws = dsa.workspace(dsa.OP_SPARSE_MLA, batch, 2048, 128)
-        dsa.sparse_mla(batch, t["q_mla"], t["latent"], idx_d, 2048, x.sm_scale, out_ref, lse_ref, ws)
+        out_ref = torch.empty((b.total_q, H, 512), dtype=torch.bfloat16, device="cuda")
+        lse_ref = torch.empty((b.total_q, H), dtype=torch.float32, device="cuda")
+        ws = dsa.workspace(dsa.OP_SPARSE_MLA, batch, k, H)
+        dsa.sparse_mla(batch, t["q_mla"], t["latent"], idx_d, k, x.sm_scale, out_ref, lse_ref, ws)
         dsa.check_device_error(ws)
         out = torch.full_like(out_ref, float("nan"))
         lse = torch.full_like(lse_ref, float("nan"))
-        assert _no_alloc(batch, t["q_mla"], t["latent"], idx_d, 2048, x.sm_scale, out, lse) == 0
+        assert _no_alloc(batch, t["q_mla"], t["latent"], idx_d, k, x.sm_scale, out, lse) == 0
         torch.cuda.synchronize()
+        check_mla(x, out.float().cpu().numpy(), lse.cpu().numpy(), idx, rows)
         _compare(out, lse, out_ref, lse_ref)
         results.append(out)
     assert not torch.equal(results[0], results[1])
+
+
+@pytest.mark.gpu
+def test_no_alloc_split_decode_two_calls():
+    # decode-shaped batch: few tokens, so the selection is split over several
+    # CTA pairs and the partial results go through the scratch array
+    x = make_inputs(custom_workload("noalloc", [4100, 3000, 5000, 2600, 6100, 3333, 4444, 2900],
+                                    [1] * 8, k_sel=2048, n_heads=128), seed=21)
+    _, batch = _setup(x)
+    assert dsa.workspace_size(dsa.OP_SPARSE_MLA, batch, 2048, 128) > 256   # the split path is taken
+    _two_calls(x, seed=5)
+
+
+@pytest.mark.gpu
+def test_no_alloc_unsplit_prefill_two_calls():
+    # prefill-shaped batch: one CTA pair per token, no partial results; here
+    # dsa_sparse_mla would gather from an fp16 copy of the cache while the
+    # no-alloc entry point gathers bf16 rows -- both within the tolerances
+    x = make_inputs("tiny_prefill_512", seed=22)
+    _, batch = _setup(x)
+    assert dsa.workspace_size(dsa.OP_SPARSE_MLA, batch, x.k_sel, x.n_heads) >= 256 + x.batch.total_keys * 1152
+    _two_calls(x, seed=6)
+
+
+@pytest.mark.gpu
+def test_no_alloc_out_of_range_sequence_leaves_no_stale_rows():
+    # A first call fills the scratch array with split partials.  The second
+    # call's batch gives one sequence a kv_start that runs past the cache: the
+    # kernel's own bounds check skips that sequence (no access through it) and
+    # its row must come out as out = 0, lse = -inf -- not as the first call's
+    # partials merged again.  The other rows are checked against the oracle.
+    x = make_inputs(custom_workload("noalloc_bad", [4100, 3000, 5000, 2600], [1] * 4, k_sel=2048, n_heads=128),
+                    seed=23)
+    t, batch = _setup(x)
+    b = x.batch
+    rng = np.random.default_rng(7)
+    idx = _random_selection(x, rng, n_drop=0)
+    idx_d = torch.from_numpy(idx).cuda()
+    out = torch.empty((b.total_q, 128, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((b.total_q, 128), dtype=torch.float32, device="cuda")
+    assert _no_alloc(batch, t["q_mla"], t["latent"], idx_d, 2048, x.sm_scale, out, lse) == 0
+    torch.cuda.synchronize()
+    bad = 2
+    ks = t["kv_start"].clone()
+    ks[bad] = b.total_keys - 100              # kv_start + kv_len > total_keys
+    batch2 = dsa.Batch(t["cu_q"], t["kv_len"], ks, b.total_q, b.max_q_per_seq, b.max_kv_len, b.total_keys)
+    out.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    assert _no_alloc(batch2, t["q_mla"], t["latent"], idx_d, 2048, x.sm_scale, out, lse) == 0
+    torch.cuda.synchronize()
+    oh, lh = out.float().cpu().numpy(), lse.cpu().numpy()
+    assert np.all(oh[bad] == 0) and np.all(np.isneginf(lh[bad]))
+    good = [r for r in range(b.total_q) if r != bad]
+    check_mla(x, oh[good], lh[good], idx[good], good)
 
 
 def test_no_alloc_scratch_covers_every_split_batch():
