@@ -80,7 +80,8 @@ typedef enum {
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA = 2,
   DSA_OP_FORWARD = 3,
-  DSA_OP_CACHE_WRITE = 4
+  DSA_OP_CACHE_WRITE = 4,
+  DSA_OP_INDEXER_TOPK = 5
 } dsa_op_t;
 
 /* Host struct describing a ragged batch; the three arrays are DEVICE memory. */
@@ -103,9 +104,11 @@ typedef struct {
 #define DSA_MAX_K_SEL 2048
 
 /* Bytes of device workspace the call `op` needs for this batch.  Returns 0
- * when the arguments are invalid.  For DSA_OP_FORWARD this includes the
- * [total_q, ld] fp32 score matrix, ld = max_kv_len rounded up to 4.  For
- * DSA_OP_TOPK (and inside DSA_OP_FORWARD) rows longer than 32768 positions
+ * when the arguments are invalid.  For DSA_OP_FORWARD and DSA_OP_INDEXER_TOPK
+ * this includes the [total_q, ld] fp32 score matrix, ld = max_kv_len rounded
+ * up to 4 -- except for decode batches (at most 2 query tokens per sequence,
+ * rows the fused kernel's clusters hold), whose scores never leave the chip.
+ * For DSA_OP_TOPK (and the unfused forward) rows longer than 32768 positions
  * with k_sel a multiple of 4 add 8 * k_sel bytes per row and 32768-position
  * segment: the candidates of the two-phase selection. */
 DSA_API size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads);
@@ -130,6 +133,21 @@ DSA_API dsa_status_t dsa_indexer_scores(const dsa_batch_t* batch, const void* q_
 DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int64_t ld_scores, int32_t k_sel,
                       int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Indexer scores and top-k in one call: `idx` as dsa_topk returns it for the
+ * scores dsa_indexer_scores computes, bit for bit.  For decode batches (at
+ * most 2 query tokens per sequence, rows of up to 16 x 16384 positions) one
+ * fused kernel does both ("DeepSeek V3.2 稀疏注意力", what happens in prefill
+ * and decode: score tile by tile, keep local candidates, merge, and hand the
+ * selection to sparse MLA without writing the score matrix to HBM): a
+ * cluster of CTAs per sequence scores one contiguous key chunk per CTA into
+ * shared memory and selects with an exact radix select whose histograms are
+ * reduced across the cluster.  Other batches run the two kernels with the
+ * scores in `ws`.  Arguments as for dsa_indexer_scores and dsa_topk; ws of
+ * dsa_workspace_size(DSA_OP_INDEXER_TOPK, ...) bytes. */
+DSA_API dsa_status_t dsa_indexer_topk(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale,
+                                      const float* w, const void* k_fp8, const float* k_scale, int32_t k_sel,
+                                      int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* Sparse MLA (MQA mode).
  *   q    [total_q, n_heads, 576] bf16        kv [total_keys, 576] bf16 latent cache
  *   idx  [total_q, k_sel] int32 positions; entries < 0 or >= kv_len are skipped
@@ -153,8 +171,9 @@ DSA_API dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int
                             const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
                             size_t ws_bytes, dsa_stream_t stream);
 
-/* The whole hot path: indexer scores (kept in ws), top-k into `idx`, sparse
- * MLA into `out`/`lse`.  Arguments as above. */
+/* The whole hot path: indexer scores and top-k into `idx` (as
+ * dsa_indexer_topk: fused on chip for decode batches, else with the scores
+ * kept in ws), sparse MLA into `out`/`lse`.  Arguments as above. */
 DSA_API dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale, const float* w,
                          const void* k_fp8, const float* k_scale, int32_t k_sel, const void* q, int32_t n_heads,
                          const void* kv, float sm_scale, int32_t* idx, void* out, float* lse, void* ws,
@@ -242,8 +261,9 @@ DSA_API dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* k, co
  * receive the kernel site id and detail recorded with the error. */
 DSA_API dsa_status_t dsa_check_device_error(void* ws, dsa_stream_t stream, uint32_t* site, uint32_t* info);
 
-/* Kernel launches one dsa_forward call makes for this batch: the indexer, the
- * top-k (two for rows longer than 32768 positions with k_sel a multiple of 4),
+/* Kernel launches one dsa_forward call makes for this batch: the indexer and
+ * the top-k (one fused launch for decode batches; otherwise one plus one, or
+ * two for rows longer than 32768 positions with k_sel a multiple of 4),
  * the fp16 copy of the latent cache when the selections reuse its rows often,
  * the sparse MLA, and the merge of split selections.  0 when the arguments are
  * invalid.  Host-only; for accounting and profiling. */

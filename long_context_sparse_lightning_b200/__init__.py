@@ -22,7 +22,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdsa.so")
 
-OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_CACHE_WRITE = 0, 1, 2, 3, 4
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_CACHE_WRITE, OP_INDEXER_TOPK = 0, 1, 2, 3, 4, 5
 INDEX_HEADS, INDEX_DIM, LATENT_DIM, VALUE_DIM, MAX_K_SEL = 64, 128, 576, 512, 2048
 
 STATUS = {
@@ -40,6 +40,7 @@ EXPORTS = [
     "dsa_workspace_size",
     "dsa_indexer_scores",
     "dsa_topk",
+    "dsa_indexer_topk",
     "dsa_sparse_mla",
     "dsa_forward",
     "dsa_sparse_mla_no_alloc",
@@ -90,6 +91,8 @@ def _lib():
         lib.dsa_indexer_scores.restype = ctypes.c_int
         lib.dsa_topk.argtypes = [BP, P, I64, I32, P, P, SZ, P]
         lib.dsa_topk.restype = ctypes.c_int
+        lib.dsa_indexer_topk.argtypes = [BP, P, P, P, P, P, I32, P, P, SZ, P]
+        lib.dsa_indexer_topk.restype = ctypes.c_int
         lib.dsa_sparse_mla.argtypes = [BP, P, I32, P, P, I32, F, P, P, P, SZ, P]
         lib.dsa_sparse_mla.restype = ctypes.c_int
         lib.dsa_forward.argtypes = [BP, P, P, P, P, P, I32, P, I32, P, F, P, P, P, P, SZ, P]
@@ -197,6 +200,12 @@ def indexer_scores(batch: Batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ws, 
 def topk(batch: Batch, scores, k_sel: int, idx, ws, stream=None):
     _check(_lib().dsa_topk(batch.ref, _ptr(scores), scores.shape[-1], k_sel, _ptr(idx), _ptr(ws), ws.numel(),
                            _stream(stream)), "dsa_topk")
+
+
+def indexer_topk(batch: Batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel: int, idx, ws, stream=None):
+    """Indexer scores and top-k in one call (fused on chip for decode batches)."""
+    _check(_lib().dsa_indexer_topk(batch.ref, _ptr(q_fp8), _ptr(q_scale), _ptr(w), _ptr(k_fp8), _ptr(k_scale), k_sel,
+                                   _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
 
 
 def sparse_mla(batch: Batch, q, kv, idx, k_sel: int, sm_scale: float, out, lse, ws, stream=None):

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdsa.so")
 SOURCES = ["api.cu", "api_no_alloc.cu", "indexer_sm100.cu", "topk.cu", "sparse_mla_sm100.cu", "prep.cu"]
-HEADERS = ["ptx.cuh", "kernels.cuh"]
+HEADERS = ["ptx.cuh", "kernels.cuh", "select.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

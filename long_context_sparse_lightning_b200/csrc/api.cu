@@ -84,6 +84,11 @@ dsa_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 int64_t forward_ld(const dsa_batch_t* b) { return static_cast<int64_t>(align_up(b->max_kv_len, 4)); }
 
+// the [total_q, ld] fp32 score matrix the unfused indexer -> top-k keeps in ws
+size_t scores_bytes(const dsa_batch_t* b) {
+  return align_up(static_cast<size_t>(b->total_q) * forward_ld(b) * sizeof(float), 256);
+}
+
 struct MlaSplit {
   int nsplit;
   int keys_per_split;
@@ -149,6 +154,44 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   p.budget = wait_budget();
   const dim3 grid((tiles + tpc - 1) / tpc, qblocks, b->num_seqs);
   return dsa::launch_indexer(tok, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// The fused decode indexer + top-k applies (CTAs per cluster), or 0.
+int fused_cluster(const dsa_batch_t* b) {
+  return dsa::indexer_topk_cluster(b->max_q_per_seq, b->num_seqs, b->max_kv_len);
+}
+
+dsa_status_t run_indexer_topk(const dsa_batch_t* b, const void* q_fp8, const float* q_scale, const float* w,
+                              const void* k_fp8, const float* k_scale, int k_sel, int32_t* idx, uint32_t* err,
+                              cudaStream_t stream) {
+  const int tok = b->max_q_per_seq;     // 1 or 2
+  const int cl = fused_cluster(b);
+  if (cl < 1) return DSA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk;
+  if (!make_tmap_2d(&tq, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_q) * 64, 128,
+                    dsa::indexer_box_rows_q(tok), 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128, 128,
+                    128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  dsa::IndexerTopkParams p;
+  p.ix.cu_q = b->cu_q;
+  p.ix.kv_len = b->kv_len;
+  p.ix.kv_start = b->kv_start;
+  p.ix.q_scale = q_scale;
+  p.ix.w = w;
+  p.ix.k_scale = k_scale;
+  p.ix.scores = nullptr;
+  p.ix.ld = 0;
+  p.ix.total_keys = b->total_keys;
+  p.ix.tiles_per_chunk = 0;
+  p.ix.num_qblocks = 1;
+  p.ix.err = err;
+  p.ix.budget = wait_budget();
+  p.k_sel = k_sel;
+  p.idx = idx;
+  p.max_kv_len = b->max_kv_len;
+  const dim3 grid(static_cast<unsigned>(cl), 1, static_cast<unsigned>(b->num_seqs));
+  return dsa::launch_indexer_topk(tok, cl, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // candidate buffers of the two-phase top-k (rows longer than 32768 positions)
@@ -284,11 +327,15 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, 
       return kHeaderBytes + mla_ws_bytes(batch, k_sel);
     case DSA_OP_CACHE_WRITE:
       return kHeaderBytes;
+    case DSA_OP_INDEXER_TOPK:
+      if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return 0;
+      if (fused_cluster(batch) > 0) return kHeaderBytes;
+      return kHeaderBytes + scores_bytes(batch) + topk_ws_bytes(batch, k_sel);
     case DSA_OP_FORWARD: {
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
-      const size_t scores = align_up(static_cast<size_t>(batch->total_q) * forward_ld(batch) * sizeof(float), 256);
+      if (fused_cluster(batch) > 0) return kHeaderBytes + mla_ws_bytes(batch, k_sel);
       // the top-k candidates and the MLA buffers are used one after the other
-      return kHeaderBytes + scores + std::max(mla_ws_bytes(batch, k_sel), topk_ws_bytes(batch, k_sel));
+      return kHeaderBytes + scores_bytes(batch) + std::max(mla_ws_bytes(batch, k_sel), topk_ws_bytes(batch, k_sel));
     }
   }
   return 0;
@@ -350,20 +397,48 @@ dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const floa
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  uint8_t* part;
+  if (fused_cluster(batch) > 0) {          // decode: scores stay on chip
+    part = base + kHeaderBytes;
+    if ((s = run_indexer_topk(batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel, idx, err, st)) != DSA_OK) return s;
+  } else {
+    const int64_t ld = forward_ld(batch);
+    float* scores = reinterpret_cast<float*>(base + kHeaderBytes);
+    part = base + kHeaderBytes + scores_bytes(batch);
+    if ((s = run_indexer(batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ld, err, st)) != DSA_OK) return s;
+    if ((s = run_topk(batch, scores, ld, k_sel, idx, part, err, st)) != DSA_OK) return s;
+  }
+  return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, part, err, st);
+}
+
+dsa_status_t dsa_indexer_topk(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale, const float* w,
+                              const void* k_fp8, const float* k_scale, int32_t k_sel, int32_t* idx, void* ws,
+                              size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer_args(batch, q_fp8, q_scale, w, k_fp8, k_scale)) != DSA_OK) return s;
+  if (idx == nullptr) return DSA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
+  const size_t need = dsa_workspace_size(DSA_OP_INDEXER_TOPK, batch, k_sel, 1);
+  if ((s = check_ws(ws, ws_bytes, need)) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  if (fused_cluster(batch) > 0)
+    return run_indexer_topk(batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel, idx, err, st);
   const int64_t ld = forward_ld(batch);
   float* scores = reinterpret_cast<float*>(base + kHeaderBytes);
-  uint8_t* part = base + kHeaderBytes + align_up(static_cast<size_t>(batch->total_q) * ld * sizeof(float), 256);
   if ((s = run_indexer(batch, q_fp8, q_scale, w, k_fp8, k_scale, scores, ld, err, st)) != DSA_OK) return s;
-  if ((s = run_topk(batch, scores, ld, k_sel, idx, part, err, st)) != DSA_OK) return s;
-  return run_mla(batch, q, n_heads, kv, idx, k_sel, sm_scale, out, lse, part, err, st);
+  return run_topk(batch, scores, ld, k_sel, idx, base + kHeaderBytes + scores_bytes(batch), err, st);
 }
 
 int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads) {
   if (check_batch(batch) != DSA_OK) return 0;
   if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
   if (batch->total_q == 0) return 0;
-  int32_t n = 1;                                                             // indexer
-  n += dsa::topk_segments(batch->max_kv_len, k_sel, batch->total_q).segs > 0 ? 2 : 1;
+  int32_t n = 1;                                                             // indexer (fused: + top-k)
+  if (fused_cluster(batch) == 0) n += dsa::topk_segments(batch->max_kv_len, k_sel, batch->total_q).segs > 0 ? 2 : 1;
   if (mla_copy(batch, k_sel)) n += 1;                                        // fp16 latent copy
   n += 1;                                                                    // sparse MLA
   if (mla_split(batch, k_sel).nsplit > 1) n += 1;                            // merge

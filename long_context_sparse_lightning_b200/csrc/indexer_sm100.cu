@@ -25,8 +25,11 @@
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner),
 // warps 2..17 = epilogue (four warpgroups).
+#include <atomic>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "select.cuh"
 
 namespace dsa {
 namespace {
@@ -282,6 +285,415 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ===========================================================================
+// Fused decode indexer + top-k
+//
+// "DeepSeek V3.2 稀疏注意力" (what happens in prefill and decode): score the
+// keys tile by tile, keep local candidates, merge them, and hand the selection
+// straight to sparse MLA without writing the score matrix to HBM.  Here a
+// cluster of C CTAs takes one (sequence, token group) of a decode batch: CTA r
+// scores a contiguous chunk of the row's key tiles exactly as the indexer
+// kernel above does, but keeps the scores in its shared memory; the cluster
+// then selects the row's top k with an exact radix select over
+// order-preserving keys (11/11/10-bit digits), the per-digit histograms
+// all-reduced across the cluster through distributed shared memory.  Equal
+// scores are taken in ascending position (lower position wins), so each CTA
+// gets a quota of the threshold-valued positions in rank order, and writes its
+// selected positions, ascending, at its offset in the output row -- the same
+// set and order as dsa_topk on the same scores.
+//
+// Every CTA of a cluster executes the same sequence of cluster barriers: the
+// only early exits depend on the cluster's (sequence, token group) alone, and
+// a timed-out wait inside the tile loop only records the error and leaves the
+// scores undefined, never the selection.
+// ===========================================================================
+constexpr int kRadixBins = 2048;
+
+template <int TOK>
+struct FusedCfg {
+  static_assert(TOK == 1 || TOK == 2, "decode token groups");
+  static constexpr int N = TOK * 64;                  // MMA N: the group's tokens x 64 heads
+  static constexpr int STAGES = TOK == 1 ? 8 : 4;
+  static constexpr int TMEM_COLS = kAccBufs * N;      // 256 or 512
+  static constexpr int CAPT = 16384;                  // keys one CTA holds the scores of (per token)
+  static constexpr int Q_BYTES = TOK * 64 * 128;
+  static constexpr int K_BYTES = 128 * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_S = OFF_K + STAGES * K_BYTES;
+  static constexpr int OFF_HIST = OFF_S + TOK * CAPT * 4;
+  static constexpr int OFF_W = OFF_HIST + 2 * kRadixBins * 4;
+  static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // tmem slot (4) + pad (12) | counts [TOK][2] (16) | scan scratch [32] (128) | broadcast [4] (16)
+  static constexpr int OFF_CNT = OFF_MISC + 16;
+  static constexpr int OFF_WARP = OFF_CNT + 16;
+  static constexpr int OFF_BC = OFF_WARP + 128;
+  static constexpr int SMEM = OFF_BC + 16 + 1024;
+  static_assert(OFF_K % 1024 == 0 && OFF_S % 16 == 0 && OFF_HIST % 16 == 0, "alignment");
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+// The row's top k, selected by the C CTAs of the cluster together.  CTA
+// `crank` holds the scores of positions [p0, p0 + len) in sc[0 .. len); the
+// CTAs' ranges follow each other in rank order and cover the n > k positions
+// of the row.  Writes k positions into out (ascending).  Every thread of every
+// CTA of the cluster calls it.
+__device__ void cluster_radix_topk(const float* __restrict__ sc, int len, int p0, int k, int32_t* __restrict__ out,
+                                   uint32_t* hist, uint32_t* cnt, uint32_t* s_warp, uint32_t* s_bc, int C,
+                                   uint32_t crank) {
+  constexpr int NT = kThreads;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t FULL = 0xffffffffu;
+  uint32_t prefix = 0, remaining = static_cast<uint32_t>(k);
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int width = pass == 2 ? 10 : 11;
+    const uint32_t mask = (1u << width) - 1u;
+    const int upper = shift + width;
+    // two histogram buffers: a CTA rewrites the one of pass p - 2 only after
+    // the cluster barrier of pass p - 1, which every CTA reaches after its
+    // reads of pass p - 2
+    uint32_t* hb = hist + (pass & 1) * kRadixBins;
+    for (int j = tid; j < kRadixBins; j += NT) hb[j] = 0u;
+    __syncthreads();
+    const int rounds = (len + NT - 1) / NT;
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r) {
+      const int e = r * NT + tid;
+      uint32_t key = 0;
+      bool match = false;
+      if (e < len) {
+        key = order_key(sc[e]);
+        match = upper >= 32 || (key >> upper) == prefix;
+      }
+      const uint32_t digit = (key >> shift) & mask;
+      const uint32_t active = __ballot_sync(FULL, match);
+      if (match) {
+        const uint32_t peers = __match_any_sync(active, digit);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hb[digit], static_cast<uint32_t>(__popc(peers)));
+      }
+    }
+    __syncthreads();
+    cluster_sync();          // every CTA's histogram of this pass is complete and visible
+    // cluster-wide counts of bins 2047 - (4 tid + j), j = 0..3 (descending digits)
+    uint32_t v[4] = {0u, 0u, 0u, 0u};
+    if (tid < kRadixBins / 4) {
+      const uint32_t a = smem_u32(hb + kRadixBins - 4 - 4 * tid);
+      for (int r = 0; r < C; ++r) {
+        const uint4 h = ld_shared_cluster_v4(mapa_shared(a, static_cast<uint32_t>(r)));
+        v[0] += h.w;
+        v[1] += h.z;
+        v[2] += h.y;
+        v[3] += h.x;
+      }
+    }
+    uint32_t total;
+    uint32_t above = block_excl_scan<NT>(v[0] + v[1] + v[2] + v[3], s_warp, total);
+    // the digit d with count(digits above d) < remaining <= count(digits >= d)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (above < remaining && above + v[j] >= remaining) {
+        s_bc[0] = static_cast<uint32_t>(kRadixBins - 1 - (4 * tid + j));
+        s_bc[1] = above;
+      }
+      above += v[j];
+    }
+    __syncthreads();
+    prefix = (prefix << width) | s_bc[0];
+    remaining -= s_bc[1];
+    __syncthreads();
+  }
+  // T = the k-th largest key; `remaining` positions of key T are needed, the
+  // lowest positions first.  Each thread takes a contiguous run of positions
+  // (odd length: consecutive lanes hit different banks).
+  const uint32_t T = prefix;
+  const int seg = ((len + NT - 1) / NT) | 1;
+  const int e0 = min(tid * seg, len), e1 = min(e0 + seg, len);
+  uint32_t gt = 0, eq = 0;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t key = order_key(sc[e]);
+    gt += key > T;
+    eq += key == T;
+  }
+  uint32_t tot;
+  const uint32_t off = block_excl_scan<NT>((gt << 16) | eq, s_warp, tot);   // per-CTA counts < 2^16
+  if (tid == 0) {
+    cnt[0] = tot >> 16;
+    cnt[1] = tot & 0xFFFFu;
+  }
+  __syncthreads();
+  cluster_sync();            // every CTA's counts are visible
+  if (tid == 0) {
+    // ties go to the lower ranks (lower positions) first
+    uint32_t rem = remaining, base = 0;
+    for (uint32_t r = 0; r < crank; ++r) {
+      const uint2 c = ld_shared_cluster_v2(mapa_shared(smem_u32(cnt), r));
+      const uint32_t q = min(rem, c.y);
+      rem -= q;
+      base += c.x + q;
+    }
+    s_bc[2] = min(rem, cnt[1]);
+    s_bc[3] = base;
+  }
+  __syncthreads();
+  const uint32_t quota = s_bc[2];
+  int32_t* dst = out + s_bc[3];
+  uint32_t o_gt = off >> 16, o_eq = off & 0xFFFFu;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t key = order_key(sc[e]);
+    if (key > T) {
+      dst[o_gt + min(o_eq, quota)] = p0 + e;
+      ++o_gt;
+    } else if (key == T) {
+      if (o_eq < quota) dst[o_gt + o_eq] = p0 + e;
+      ++o_eq;
+    }
+  }
+  __syncthreads();           // s_bc / s_warp are reused by the next row
+}
+
+template <int TOK>
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_topk_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const IndexerTopkParams fp) {
+  using C = FusedCfg<TOK>;
+  const IndexerParams& p = fp.ix;
+  extern __shared__ uint8_t smem_raw[];
+
+  // ---- work unit: sequence b, token group, this CTA's chunk of key tiles.
+  // Every early exit below depends on (b, group) only: the whole cluster
+  // takes it together. ----
+  const uint32_t crank = cluster_ctarank();
+  const int ncl = static_cast<int>(gridDim.x);         // CTAs per cluster (the cluster spans x)
+  const int b = blockIdx.z;
+  const int qblock = static_cast<int>(blockIdx.y);
+  const int q0 = __ldg(&p.cu_q[b]);
+  const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
+  const int kv = __ldg(&p.kv_len[b]);
+  const int first = qblock * TOK;
+  if (first >= q_len) return;
+  const int64_t kstart = __ldg(&p.kv_start[b]);
+  if (q_len > kv || kv > fp.max_kv_len || kstart < 0 || kstart + kv > p.total_keys) {
+    if (threadIdx.x == 0 && crank == 0) report_error(p.err, kDevErrBounds, 151, b);
+    return;
+  }
+  const int ntok = min(TOK, q_len - first);
+  const int t_first = kv - q_len + first;
+  const int t_last = t_first + ntok - 1;
+  const int tiles_total = (t_last + 1 + 127) / 128;
+  const int tpc = (tiles_total + ncl - 1) / ncl;       // <= CAPT / 128 (checked on the host via max_kv_len)
+  const int tile_begin = min(static_cast<int>(crank) * tpc, tiles_total);
+  const int n_tiles = min(tile_begin + tpc, tiles_total) - tile_begin;   // may be 0
+  const int p0 = tile_begin * 128;
+  const int row0 = q0 + first;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = sm + C::OFF_Q;
+  uint8_t* sK = sm + C::OFF_K;
+  float* sS = reinterpret_cast<float*>(sm + C::OFF_S);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sm + C::OFF_HIST);
+  float* sW = reinterpret_cast<float*>(sm + C::OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* q_full = bars + 2 * C::STAGES;
+  uint64_t* acc_full = q_full + 1;
+  uint64_t* acc_empty = q_full + 1 + kAccBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(sm + C::OFF_CNT);
+  uint32_t* s_warp = reinterpret_cast<uint32_t*>(sm + C::OFF_WARP);
+  uint32_t* s_bc = reinterpret_cast<uint32_t*>(sm + C::OFF_BC);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  for (int i = threadIdx.x; i < TOK * 64; i += kThreads) {
+    const int tk = i >> 6;
+    float v = 0.f;
+    if (tk < ntok) {
+      const int64_t o = static_cast<int64_t>(row0 + tk) * 64 + (i & 63);
+      v = __ldg(&p.w[o]) * __ldg(&p.q_scale[o]);
+    }
+    sW[i] = v;
+  }
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kAccBufs; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer --
+    if (elect_one()) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      tma_load_2d(sQ, &tmap_q, q_full, 0, row0 * 64);
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 160, it);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], C::K_BYTES);
+        tma_load_2d(sK + s * C::K_BYTES, &tmap_k, &full[s], 0,
+                    static_cast<int32_t>(kstart + static_cast<int64_t>(tile_begin + it) * 128));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer --
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_f32acc(kFmtE4M3, kFmtE4M3, 128, C::N, 0, 0);
+      bool ok = mbar_wait(q_full, 0, p.budget);
+      if (!ok) report_error(p.err, kDevErrTimeout, 161, 0);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int s = it % C::STAGES;
+        const int buf = it % kAccBufs;
+        if (!mbar_wait(&full[s], (it / C::STAGES) & 1, p.budget) ||
+            !mbar_wait(&acc_empty[buf], ((it / kAccBufs) & 1) ^ 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 162, it);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sK + s * C::K_BYTES);
+        const uint32_t b_base = smem_u32(sQ);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          umma_e4m3(tmem + buf * C::N, smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B),
+                    smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&acc_full[buf]);
+        umma_commit(&empty[s]);
+      }
+    }
+  } else {
+    // --------------------------------------------------- epilogue --
+    // as in the indexer kernel, but each score goes to this CTA's chunk in
+    // shared memory (a warp stores 32 consecutive floats)
+    const int ew = static_cast<int>(warp) - 2;
+    const int g = ew >> 2;
+    const uint32_t quarter = warp & 3u;
+    const int key_in_tile = static_cast<int>(quarter * 32 + lane);
+    const uint32_t lane_addr = (quarter * 32u) << 16;
+    auto key_scale = [&](int it) {
+      const int s = (tile_begin + it) * 128 + key_in_tile;
+      return (it < n_tiles && s < kv) ? __ldg(&p.k_scale[kstart + s]) : 0.f;
+    };
+    float ks_next = key_scale(g);
+    for (int it = g; it < n_tiles; it += kAccBufs) {
+      const float ks = ks_next;
+      ks_next = key_scale(it + kAccBufs);
+      if (!mbar_wait(&acc_full[g], (it / kAccBufs) & 1, p.budget)) {
+        report_error(p.err, kDevErrTimeout, 170, it);
+        break;
+      }
+      tc_fence_after();
+      const int e = it * 128 + key_in_tile;             // chunk-local position
+#pragma unroll 1
+      for (int tk = 0; tk < TOK; ++tk) {
+        uint32_t ra[32], rb[32];
+        const uint32_t taddr = tmem + lane_addr + static_cast<uint32_t>(g * C::N + tk * 64);
+        tmem_ld32(taddr, ra);
+        tmem_ld32(taddr + 32, rb);
+        tmem_ld_wait();
+        const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(sW + tk * 64);
+        unsigned long long a01 = 0ull, a23 = 0ull;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const ulonglong2 wv = w2[j];
+          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(ra[4 * j + 0]), 0.f),
+                                  fmaxf(__uint_as_float(ra[4 * j + 1]), 0.f)), a01);
+          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(ra[4 * j + 2]), 0.f),
+                                  fmaxf(__uint_as_float(ra[4 * j + 3]), 0.f)), a23);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const ulonglong2 wv = w2[8 + j];
+          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(rb[4 * j + 0]), 0.f),
+                                  fmaxf(__uint_as_float(rb[4 * j + 1]), 0.f)), a01);
+          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(rb[4 * j + 2]), 0.f),
+                                  fmaxf(__uint_as_float(rb[4 * j + 3]), 0.f)), a23);
+        }
+        const float2 s01 = unpack2(a01), s23 = unpack2(a23);
+        sS[tk * C::CAPT + e] = ((s01.x + s01.y) + (s23.x + s23.y)) * ks;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[g]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();           // every score of the chunk is in shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+
+  // ---- selection, token by token ----
+  const int k = fp.k_sel;
+#pragma unroll 1
+  for (int tk = 0; tk < ntok; ++tk) {
+    const int n = t_first + tk + 1;                  // positions 0 .. t
+    int32_t* out = fp.idx + static_cast<int64_t>(row0 + tk) * k;
+    if (n <= k) {                                     // the whole prefix, then -1 (same in every CTA)
+      if (crank == 0)
+        for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
+      continue;
+    }
+    const int len = min(max(n - p0, 0), n_tiles * 128);
+    cluster_radix_topk(sS + tk * C::CAPT, len, p0, k, out, hist, cnt + 2 * tk, s_warp, s_bc, ncl, crank);
+  }
+  cluster_sync();            // no CTA leaves while a peer may still read its shared memory
+}
+
+template <int TOK>
+cudaError_t launch_fused_tok(int cluster, dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const IndexerTopkParams& p, cudaStream_t stream) {
+  using C = FusedCfg<TOK>;
+  auto kern = indexer_topk_kernel<TOK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  if (cluster > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int TOK>
 cudaError_t launch_tok(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const IndexerParams& p,
                        cudaStream_t stream) {
@@ -316,6 +728,74 @@ int indexer_box_rows_q(int tok) {
     case 2: return IdxCfg<2>::BOXQ;
     case 4: return IdxCfg<4>::BOXQ;
     default: return IdxCfg<8>::BOXQ;
+  }
+}
+
+// Largest cluster the fused kernel of `tok` tokens can run on this device:
+// 16 (a non-portable size) when the occupancy query finds room for one such
+// cluster, else the portable 8.  Queried once per device.
+static int fused_cluster_cap(int tok) {
+  static std::atomic<int> cache[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  std::atomic<int>& slot = cache[dev][tok == 2 ? 1 : 0];
+  int v = slot.load(std::memory_order_relaxed);
+  if (v != 0) return v;
+  v = 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(16, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (tok == 2) {
+    auto kern = indexer_topk_kernel<2>;
+    cfg.dynamicSmemBytes = FusedCfg<2>::SMEM;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<2>::SMEM) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1)
+      v = 16;
+  } else {
+    auto kern = indexer_topk_kernel<1>;
+    cfg.dynamicSmemBytes = FusedCfg<1>::SMEM;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<1>::SMEM) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1)
+      v = 16;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error behind
+  slot.store(v, std::memory_order_relaxed);
+  return v;
+}
+
+int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len) {
+  if (max_q_per_seq < 1 || max_q_per_seq > 2 || num_seqs < 1 || max_kv_len < 1) return 0;
+  const int tiles = (max_kv_len + 127) / 128;
+  constexpr int cap_tiles = FusedCfg<1>::CAPT / 128;   // the same per token for both group sizes
+  static_assert(FusedCfg<1>::CAPT == FusedCfg<2>::CAPT, "one chunk capacity");
+  const int cmax = fused_cluster_cap(max_q_per_seq);
+  // enough CTAs for the row to fit (memory) and, while the grid stays within
+  // one wave, more of them for bandwidth (each CTA streams its chunk of keys)
+  int c = 1;
+  while (c <= cmax && (tiles + c - 1) / c > cap_tiles) c *= 2;
+  if (c > cmax) return 0;
+  while (2 * c <= cmax && static_cast<int64_t>(num_seqs) * 2 * c <= sm_count() && (tiles + 2 * c - 1) / (2 * c) >= 8)
+    c *= 2;
+  return c;
+}
+
+cudaError_t launch_indexer_topk(int tok, int cluster, dim3 grid, const CUtensorMap& tmap_q,
+                                const CUtensorMap& tmap_k, const IndexerTopkParams& p, cudaStream_t stream) {
+  if (cluster < 1 || cluster > 16 || static_cast<int>(grid.x) != cluster) return cudaErrorInvalidValue;
+  switch (tok) {
+    case 1: return launch_fused_tok<1>(cluster, grid, tmap_q, tmap_k, p, stream);
+    case 2: return launch_fused_tok<2>(cluster, grid, tmap_q, tmap_k, p, stream);
+    default: return cudaErrorInvalidValue;
   }
 }
 

@@ -39,6 +39,22 @@ int indexer_box_rows_q(int tok);
 cudaError_t launch_indexer(int tok, dim3 grid, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const IndexerParams& p, cudaStream_t stream);
 
+// Fused decode indexer + top-k: a cluster of CTAs per (sequence, token
+// group) scores the row's keys into shared memory, one contiguous chunk per
+// CTA, and selects the row's top k with a cluster-wide radix select; no score
+// leaves the chip.  For batches of 1-2 query tokens per sequence.
+struct IndexerTopkParams {
+  IndexerParams ix;        // scores / ld unused
+  int32_t k_sel = 0;
+  int32_t* idx = nullptr;  // [total_q, k_sel]
+  int32_t max_kv_len = 0;  // host maximum over the batch (the chunk capacity was checked against it)
+};
+// CTAs per cluster for this batch, 0 when the fused kernel does not apply
+// (more than 2 tokens per sequence, or a row too long for 16 CTAs).
+int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len);
+cudaError_t launch_indexer_topk(int tok, int cluster, dim3 grid, const CUtensorMap& tmap_q,
+                                const CUtensorMap& tmap_k, const IndexerTopkParams& p, cudaStream_t stream);
+
 // ------------------------------------------------------------------ top-k --
 struct TopkParams {
   const int32_t* cu_q;

@@ -30,6 +30,7 @@
 
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "select.cuh"
 
 namespace dsa {
 namespace {
@@ -38,47 +39,6 @@ constexpr int kBins = 2048;
 constexpr int kCandCap = 512;     // boundary-bin positions ranked pairwise
 constexpr int kSegChunks = 16;    // chunks per compaction segment: 16 x 4 flags per thread
 constexpr int kMaxK = 2048;       // largest k_sel
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u << 1) == 0u) u = 0u;     // -0 ties with +0, as in a float comparison
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
-// Exclusive prefix sum over the block, in thread order; also returns the total.
-template <int BLOCK>
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t& total) {
-  constexpr int NW = BLOCK / 32;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  uint32_t x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) s_warp[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    uint32_t w = lane < NW ? s_warp[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < NW) s_warp[lane] = w;
-  }
-  __syncthreads();
-  const uint32_t before = wid > 0 ? s_warp[wid - 1] : 0u;
-  total = s_warp[NW - 1];
-  __syncthreads();
-  return before + x - v;
-}
 
 template <int BLOCK, int CAPW>
 struct TopkShared {

@@ -114,20 +114,31 @@ def check_mla(x, out_gpu: np.ndarray, lse_gpu, idx_rows: np.ndarray, rows, max_a
     ``value_scale``: the factor the latent entries were scaled by (1 for the
     configs' N(0,1) draws).  The output is linear in the values, so the max-abs
     bound applies to the difference divided by it; the mean relative error is
-    scale-free.  ``ulp_floor``: an element may also differ by one bf16 step of
-    its reference value -- when a peaky softmax makes outputs as large as the
-    values themselves (|o| >= 4 value scales, where one bf16 step exceeds the
-    bound), an fp32 result and the fp64 one may round to neighbouring bf16
-    numbers."""
+    scale-free.  ``ulp_floor``: an element may also differ by one bf16 step --
+    when a peaky softmax makes outputs as large as the values themselves
+    (|o| >= 4 value scales, where one bf16 step exceeds the bound), an fp32
+    result and the fp64 one may round to neighbouring bf16 numbers."""
     ref = o_mla.sparse(x, idx_rows, rows)
     sum_abs = sum_ref = 0.0
     worst = 0.0
+    where = None
     for i, r in enumerate(rows):
         o, lse = ref[int(r)]
         rb = o_mla.bf16_output(o)
-        d = np.abs(out_gpu[i].astype(np.float64) - rb)
+        g = out_gpu[i].astype(np.float64)
+        d = np.abs(g - rb)
         assert np.all(np.isfinite(out_gpu[i])), f"row {r}: non-finite output"
-        worst = max(worst, float(d.max()) / value_scale)
+        dm = d / value_scale
+        if ulp_floor:
+            # one bf16 step at the larger of the two magnitudes (the two may sit
+            # on either side of a power of two)
+            big = np.maximum(np.abs(rb), np.abs(g))
+            step = np.where(big == 0, 0.0, np.ldexp(1.0, np.frexp(big)[1] - 8))
+            dm = np.where(d <= step, np.minimum(dm, max_abs), dm)
+        j = np.unravel_index(int(np.argmax(dm)), dm.shape)
+        if float(dm[j]) > worst or where is None:
+            worst = max(worst, float(dm[j]))
+            where = (int(r), tuple(int(v) for v in j), float(rb[j]), float(g[j]))
         sum_abs += float(d.sum())
         sum_ref += float(np.abs(rb).sum())
         if lse_gpu is not None:
@@ -135,7 +146,7 @@ def check_mla(x, out_gpu: np.ndarray, lse_gpu, idx_rows: np.ndarray, rows, max_a
             assert np.array_equal(np.isfinite(lse_gpu[i]), fin), f"row {r}: lse finiteness differs"
             assert np.allclose(lse_gpu[i][fin], lse[fin], rtol=1e-4, atol=2e-3), f"row {r}: lse"
     rel = sum_abs / max(sum_ref, 1e-300)
-    assert worst <= max_abs, f"max |d| = {worst}"
+    assert worst <= max_abs, f"max |d| = {worst} at (row, (head, dim), ref, gpu) = {where}"
     assert rel <= mean_rel, f"mean relative error = {rel}"
     return worst, rel
 

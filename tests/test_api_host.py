@@ -74,10 +74,29 @@ def test_forward_launch_counts():
     # one long-context sequence of many queries: + the fp16 latent copy
     pre = _host_batch(B=1, total_q=4096, max_q=4096, max_kv=32768, total_keys=32768)
     assert lib.dsa_forward_launches(ctypes.byref(pre), 2048, 128) == 4
-    # a few decode tokens at 128K: two-phase top-k and split selections + merge
+    # a few decode tokens at 128K: the fused indexer + top-k, split selections + merge
     dec = _host_batch(B=8, total_q=16, max_q=2, max_kv=131072, total_keys=8 * 131072)
-    assert lib.dsa_forward_launches(ctypes.byref(dec), 2048, 128) == 5
+    assert lib.dsa_forward_launches(ctypes.byref(dec), 2048, 128) == 3
     assert lib.dsa_forward_launches(ctypes.byref(dec), 4096, 128) == 0      # k_sel too large
+    # three query tokens per sequence: no fused kernel; two-phase top-k at 128K
+    dec3 = _host_batch(B=8, total_q=24, max_q=3, max_kv=131072, total_keys=8 * 131072)
+    assert lib.dsa_forward_launches(ctypes.byref(dec3), 2048, 128) == 5
+
+
+def test_fused_decode_workspace_holds_no_scores():
+    lib = dsa.library()
+    # decode: scores stay on chip, the indexer + top-k needs only the error word
+    dec = _host_batch(B=64, total_q=64, max_q=1, max_kv=32768, total_keys=64 * 32768)
+    assert lib.dsa_workspace_size(dsa.OP_INDEXER_TOPK, ctypes.byref(dec), 2048, 128) == 256
+    fwd = lib.dsa_workspace_size(dsa.OP_FORWARD, ctypes.byref(dec), 2048, 128)
+    assert fwd == lib.dsa_workspace_size(dsa.OP_SPARSE_MLA, ctypes.byref(dec), 2048, 128)
+    # prefill: the [total_q, ld] fp32 score matrix
+    pre = _host_batch(B=1, total_q=4096, max_q=4096, max_kv=32768, total_keys=32768)
+    n = lib.dsa_workspace_size(dsa.OP_INDEXER_TOPK, ctypes.byref(pre), 2048, 128)
+    assert n == 256 + 4096 * 32768 * 4
+    # rows too long for 16 CTAs of 16384 positions: unfused
+    huge = _host_batch(B=1, total_q=1, max_q=1, max_kv=300000, total_keys=300000)
+    assert lib.dsa_workspace_size(dsa.OP_INDEXER_TOPK, ctypes.byref(huge), 2048, 128) > 256 + 300000 * 4
 
 
 def test_rejections_happen_before_any_launch():
