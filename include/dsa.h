@@ -84,16 +84,30 @@ typedef enum {
   DSA_OP_INDEXER_TOPK = 5
 } dsa_op_t;
 
-/* Host struct describing a ragged batch; the three arrays are DEVICE memory. */
+/* Host struct describing a ragged batch; the arrays are DEVICE memory.
+ *
+ * Caches are flat (block_table == NULL: position s of sequence b is cache row
+ * kv_start[b] + s) or paged (block_table != NULL: the key, key-scale and
+ * latent caches are pools of total_keys / page_size pages of page_size rows,
+ * and position s of sequence b is pool row
+ *     block_table[b * blocks_per_seq + s / page_size] * page_size + s % page_size;
+ * kv_start is then ignored and may be NULL).  "DeepSeek V3.2 稀疏注意力" lists
+ * this logical-position -> block/offset map among what a decode kernel must
+ * define.  A page id outside [0, total_keys / page_size) is a device-side
+ * bounds error (DSA_ERR_DEVICE_BOUNDS); the row it would address is not read. */
 typedef struct {
   int32_t num_seqs;          /* B >= 1                                             */
   int32_t total_q;           /* cu_q[B]; query rows of every per-row tensor       */
   int32_t max_q_per_seq;     /* max_b q_len[b] (host copy, sizes the grids)       */
   int32_t max_kv_len;        /* max_b kv_len[b] (host copy)                       */
-  int64_t total_keys;        /* rows of the flat key / latent caches (< 2^31)     */
+  int64_t total_keys;        /* rows of the key / latent caches or pools (< 2^31) */
   const int32_t* cu_q;       /* [B+1] query-row offsets, cu_q[0] = 0              */
   const int32_t* kv_len;     /* [B] positions present, including the new queries  */
   const int64_t* kv_start;   /* [B] first flat cache row of each sequence          */
+  const int32_t* block_table;  /* [B, blocks_per_seq] page ids, or NULL (flat)     */
+  int32_t page_size;         /* paged: rows per page, a positive multiple of 64    */
+  int32_t blocks_per_seq;    /* paged: row stride of block_table,
+                                >= ceil(max_kv_len / page_size)                    */
 } dsa_batch_t;
 
 /* Fixed sizes of the hot path (the pages' indexer: 64 heads of dim 128). */
@@ -272,7 +286,8 @@ DSA_API int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, in
 /* Static description of a status code. */
 DSA_API const char* dsa_status_string(dsa_status_t status);
 
-/* ABI version (major * 100 + minor). */
+/* ABI version (major * 100 + minor); 200 added the paged-cache fields of
+ * dsa_batch_t and dsa_indexer_topk. */
 DSA_API int32_t dsa_version(void);
 
 #ifdef __cplusplus

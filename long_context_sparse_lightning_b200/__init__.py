@@ -69,6 +69,9 @@ class _BatchC(ctypes.Structure):
         ("cu_q", ctypes.c_void_p),
         ("kv_len", ctypes.c_void_p),
         ("kv_start", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32),
+        ("blocks_per_seq", ctypes.c_int32),
     ]
 
 
@@ -141,13 +144,22 @@ def _check(status: int, where: str):
 
 class Batch:
     """Ragged batch: device arrays cu_q [B+1] int32, kv_len [B] int32, kv_start [B] int64,
-    plus the host-side sizes that shape the launch grids."""
+    plus the host-side sizes that shape the launch grids.
 
-    def __init__(self, cu_q: torch.Tensor, kv_len: torch.Tensor, kv_start: torch.Tensor, total_q: int,
-                 max_q_per_seq: int, max_kv_len: int, total_keys: int):
-        if cu_q.dtype != torch.int32 or kv_len.dtype != torch.int32 or kv_start.dtype != torch.int64:
+    Paged caches: pass ``block_table`` (int32 [B, blocks_per_seq] page ids) and
+    ``page_size`` (a multiple of 64); ``kv_start`` may then be None and
+    ``total_keys`` is the pool's row count."""
+
+    def __init__(self, cu_q: torch.Tensor, kv_len: torch.Tensor, kv_start: Optional[torch.Tensor], total_q: int,
+                 max_q_per_seq: int, max_kv_len: int, total_keys: int, block_table: Optional[torch.Tensor] = None,
+                 page_size: int = 0):
+        if cu_q.dtype != torch.int32 or kv_len.dtype != torch.int32 or \
+                (kv_start is not None and kv_start.dtype != torch.int64):
             raise TypeError("cu_q/kv_len must be int32 and kv_start int64")
-        self.cu_q, self.kv_len, self.kv_start = cu_q, kv_len, kv_start
+        if block_table is not None and (block_table.dtype != torch.int32 or block_table.dim() != 2
+                                        or not block_table.is_contiguous()):
+            raise TypeError("block_table must be a contiguous int32 [num_seqs, blocks_per_seq] tensor")
+        self.cu_q, self.kv_len, self.kv_start, self.block_table = cu_q, kv_len, kv_start, block_table
         self.num_seqs = int(kv_len.shape[0])
         self.total_q = int(total_q)
         self.c = _BatchC()
@@ -158,7 +170,11 @@ class Batch:
         self.c.total_keys = int(total_keys)
         self.c.cu_q = cu_q.data_ptr()
         self.c.kv_len = kv_len.data_ptr()
-        self.c.kv_start = kv_start.data_ptr()
+        self.c.kv_start = kv_start.data_ptr() if kv_start is not None else None
+        if block_table is not None:
+            self.c.block_table = block_table.data_ptr()
+            self.c.page_size = int(page_size)
+            self.c.blocks_per_seq = int(block_table.shape[1])
 
     @staticmethod
     def from_host(cu_q, kv_len, kv_start, device="cuda", total_keys: Optional[int] = None):

@@ -66,7 +66,17 @@ dsa_status_t check_batch(const dsa_batch_t* b) {
   if (b->num_seqs < 1 || b->num_seqs > 65535 || b->total_q < 0 || b->max_q_per_seq < 0 || b->max_kv_len < 0 ||
       b->total_keys < 0)
     return DSA_ERR_INVALID_ARG;
-  if (b->cu_q == nullptr || b->kv_len == nullptr || b->kv_start == nullptr) return DSA_ERR_INVALID_ARG;
+  if (b->cu_q == nullptr || b->kv_len == nullptr) return DSA_ERR_INVALID_ARG;
+  if (b->block_table == nullptr) {
+    if (b->kv_start == nullptr) return DSA_ERR_INVALID_ARG;
+  } else {
+    // pages of a multiple of 64 rows (the key tiles load as 64-row halves), a
+    // table row long enough for the longest sequence, a whole number of pages
+    if (b->page_size < 64 || (b->page_size % 64) != 0 || b->blocks_per_seq < 1) return DSA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(b->blocks_per_seq) * b->page_size < b->max_kv_len) return DSA_ERR_INVALID_ARG;
+    if (b->total_keys % b->page_size != 0) return DSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(b->block_table) & 3u) != 0) return DSA_ERR_INVALID_ARG;
+  }
   if (b->total_q > 0 && (b->max_q_per_seq < 1 || b->max_kv_len < b->max_q_per_seq || b->total_keys < 1))
     return DSA_ERR_INVALID_ARG;
   if (b->max_q_per_seq > b->total_q || static_cast<int64_t>(b->max_kv_len) > b->total_keys)
@@ -75,6 +85,21 @@ dsa_status_t check_batch(const dsa_batch_t* b) {
     return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
+
+dsa::PageTable page_table(const dsa_batch_t* b) {
+  dsa::PageTable pt;
+  if (b->block_table != nullptr) {
+    pt.table = b->block_table;
+    pt.page = b->page_size;
+    pt.stride = b->blocks_per_seq;
+    pt.num_pages = static_cast<int32_t>(b->total_keys / b->page_size);
+  }
+  return pt;
+}
+
+// key-tile box height of the indexer's key-cache descriptor: whole 128-key
+// tiles (flat) or 64-row halves, one per page run (paged)
+uint32_t k_box_rows(const dsa_batch_t* b) { return b->block_table != nullptr ? 64 : 128; }
 
 dsa_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (ws == nullptr || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
@@ -124,8 +149,8 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   CUtensorMap tq, tk;
   if (!make_tmap_2d(&tq, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_q) * 64, 128,
                     dsa::indexer_box_rows_q(tok), 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128, 128,
-                    128, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128,
+                    k_box_rows(b), 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   const int qblocks = (b->max_q_per_seq + tok - 1) / tok;
   if (qblocks > 65535) return DSA_ERR_UNSUPPORTED;
@@ -152,6 +177,7 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   p.num_qblocks = qblocks;
   p.err = err;
   p.budget = wait_budget();
+  p.pt = page_table(b);
   const dim3 grid((tiles + tpc - 1) / tpc, qblocks, b->num_seqs);
   return dsa::launch_indexer(tok, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -170,8 +196,8 @@ dsa_status_t run_indexer_topk(const dsa_batch_t* b, const void* q_fp8, const flo
   CUtensorMap tq, tk;
   if (!make_tmap_2d(&tq, q_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_q) * 64, 128,
                     dsa::indexer_box_rows_q(tok), 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128, 128,
-                    128, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap_2d(&tk, k_fp8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(b->total_keys), 128,
+                    k_box_rows(b), 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   dsa::IndexerTopkParams p;
   p.ix.cu_q = b->cu_q;
@@ -187,6 +213,7 @@ dsa_status_t run_indexer_topk(const dsa_batch_t* b, const void* q_fp8, const flo
   p.ix.num_qblocks = 1;
   p.ix.err = err;
   p.ix.budget = wait_budget();
+  p.ix.pt = page_table(b);
   p.k_sel = k_sel;
   p.idx = idx;
   p.max_kv_len = b->max_kv_len;
@@ -238,6 +265,7 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   p.idx = idx;
   p.total_keys = b->total_keys;
   p.total_q = b->total_q;
+  p.pt = page_table(b);
   p.k_sel = k_sel;
   p.n_heads = n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
@@ -294,6 +322,9 @@ dsa_status_t check_mla_args(const void* q, int n_heads, const void* kv, int k_se
 }  // namespace
 
 namespace dsa {
+dsa_status_t validate_batch(const dsa_batch_t* b) { return check_batch(b); }
+PageTable batch_pages(const dsa_batch_t* b) { return page_table(b); }
+
 long long wait_budget() {
   const char* s = std::getenv("DSA_WAIT_BUDGET_CYCLES");
   if (s != nullptr) {
@@ -466,8 +497,9 @@ dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* k, const void
   if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
   if (batch->total_q == 0) return DSA_OK;
   return dsa::launch_cache_write(batch->num_seqs, batch->max_q_per_seq, batch->total_q, batch->total_keys,
-                                 batch->cu_q, batch->kv_len, batch->kv_start, k, latent, k_cache, k_scale,
-                                 latent_cache, static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream)) ==
+                                 batch->cu_q, batch->kv_len, batch->kv_start, page_table(batch), k, latent, k_cache,
+                                 k_scale, latent_cache, static_cast<uint32_t*>(ws),
+                                 reinterpret_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? DSA_OK
              : DSA_ERR_CUDA;
@@ -505,6 +537,6 @@ const char* dsa_status_string(dsa_status_t status) {
   return "unknown status";
 }
 
-int32_t dsa_version(void) { return 100; }
+int32_t dsa_version(void) { return 200; }
 
 }  // extern "C"

@@ -59,15 +59,8 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
                                                 const int32_t* idx, int32_t k_sel, float sm_scale, void* out,
                                                 float* lse, dsa_stream_t stream) {
   // ---- argument checks, the same rules as dsa_sparse_mla ----
-  if (b == nullptr || b->num_seqs < 1 || b->num_seqs > 65535 || b->total_q < 0 || b->max_q_per_seq < 0 ||
-      b->max_kv_len < 0 || b->total_keys < 0 || b->cu_q == nullptr || b->kv_len == nullptr || b->kv_start == nullptr)
-    return DSA_ERR_INVALID_ARG;
-  if (b->total_q > 0 && (b->max_q_per_seq < 1 || b->max_kv_len < b->max_q_per_seq || b->total_keys < 1))
-    return DSA_ERR_INVALID_ARG;
-  if (b->max_q_per_seq > b->total_q || static_cast<int64_t>(b->max_kv_len) > b->total_keys)
-    return DSA_ERR_INVALID_ARG;
-  if (b->total_keys >= (int64_t(1) << 31) || static_cast<int64_t>(b->total_q) * 128 >= (int64_t(1) << 31))
-    return DSA_ERR_UNSUPPORTED;
+  const dsa_status_t bs = dsa::validate_batch(b);
+  if (bs != DSA_OK) return bs;
   auto misaligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
   if (q == nullptr || kv == nullptr || out == nullptr || idx == nullptr) return DSA_ERR_INVALID_ARG;
   if (misaligned(q) || misaligned(kv) || misaligned(out)) return DSA_ERR_INVALID_ARG;
@@ -102,6 +95,7 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   p.idx = idx;
   p.total_keys = b->total_keys;
   p.total_q = b->total_q;
+  p.pt = dsa::batch_pages(b);
   p.k_sel = k_sel;
   p.n_heads = n_heads;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);

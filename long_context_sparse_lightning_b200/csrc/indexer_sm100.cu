@@ -54,7 +54,8 @@ struct IdxCfg {
   static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-byte alignment
+  static constexpr int OFF_PAGE = OFF_MISC + 16;      // paged caches: pool row of each 64-key half tile
+  static constexpr int SMEM = OFF_PAGE + 1024;        // + slack for 1024-byte alignment (+ 8 B per tile when paged)
   static_assert(OFF_K % 1024 == 0 && K_BYTES % 1024 == 0, "swizzle-128 tiles need 1024-byte alignment");
 };
 
@@ -76,6 +77,47 @@ __device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsign
   return d;
 }
 
+// Paged caches: the pool row of every 64-key half of this CTA's key tiles
+// (positions past the sequence, or a page id outside the pool, get
+// total_keys: a TMA box there reads zeros and no key scale is loaded).
+__device__ __forceinline__ void stage_half_tile_rows(const PageTable& pt, int b, int kv, int tile_begin, int n_tiles,
+                                                     int64_t total_keys, int32_t* sPage, uint32_t* err) {
+  for (int i = threadIdx.x; i < 2 * n_tiles; i += blockDim.x) {
+    const int s = tile_begin * 128 + i * 64;
+    int64_t row = total_keys;
+    if (s < kv) {
+      row = cache_row(pt, b, 0, s);
+      if (row < 0) {
+        report_error(err, kDevErrBounds, 103, b);
+        row = total_keys;
+      }
+    }
+    sPage[i] = static_cast<int32_t>(row);
+  }
+}
+
+// One 128-key tile of the key cache into a stage: one 128-row box (flat), or
+// two 64-row boxes from their pages -- stacked, they form the same 128-byte
+// swizzled layout (the swizzle repeats every 8 rows).
+__device__ __forceinline__ void load_k_tile(uint8_t* dst, const CUtensorMap* tmap, uint64_t* bar, bool paged,
+                                            const int32_t* sPage, int it, int64_t flat_row) {
+  if (paged) {
+    tma_load_2d(dst, tmap, bar, 0, sPage[2 * it]);
+    tma_load_2d(dst + 8192, tmap, bar, 0, sPage[2 * it + 1]);
+  } else {
+    tma_load_2d(dst, tmap, bar, 0, static_cast<int32_t>(flat_row));
+  }
+}
+
+// Scale of the key at position `flat_row - kstart` (flat) or at offset
+// key_in_tile of local tile `it` (paged).
+__device__ __forceinline__ float scale_of_key(const float* k_scale, bool paged, const int32_t* sPage, int it,
+                                              int key_in_tile, int64_t flat_row, int64_t total_keys) {
+  if (!paged) return __ldg(&k_scale[flat_row]);
+  const int64_t base = sPage[2 * it + (key_in_tile >> 6)];
+  return base < total_keys ? __ldg(&k_scale[base + (key_in_tile & 63)]) : 0.f;
+}
+
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -92,8 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kv = __ldg(&p.kv_len[b]);
   const int first = qblock * TOK;
   if (first >= q_len) return;
-  const int64_t kstart = __ldg(&p.kv_start[b]);
-  if (q_len > kv || kv > p.ld || kstart < 0 || kstart + kv > p.total_keys) {
+  const int64_t kstart = seq_start(p.pt, p.kv_start, b);
+  if (q_len > kv || kv > p.ld || !seq_rows_ok(p.pt, kstart, kv, p.total_keys)) {
     if (threadIdx.x == 0) report_error(p.err, kDevErrBounds, 101, b);
     return;
   }
@@ -103,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles_total = (t_last + 1 + 127) / 128;
   const int tile_begin = static_cast<int>(blockIdx.x) * p.tiles_per_chunk;
   if (tile_begin >= tiles_total) return;
+  const bool paged = p.pt.table != nullptr;
   const int n_tiles = min(tile_begin + p.tiles_per_chunk, tiles_total) - tile_begin;
   const int row0 = q0 + first;
 
@@ -119,10 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = q_full + 1;               // [kAccBufs]
   uint64_t* acc_empty = q_full + 1 + kAccBufs;    // [kAccBufs]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  int32_t* sPage = reinterpret_cast<int32_t*>(sm + C::OFF_PAGE);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
+  if (paged) stage_half_tile_rows(p.pt, b, kv, tile_begin, n_tiles, p.total_keys, sPage, p.err);
   // w' = w * q_scale for this CTA's tokens (0 for rows past the sequence)
   for (int i = threadIdx.x; i < TOK * 64; i += kThreads) {
     const int tk = i >> 6;
@@ -172,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&full[s], C::K_BYTES);
-        tma_load_2d(sK + s * C::K_BYTES, &tmap_k, &full[s], 0,
-                    static_cast<int32_t>(kstart + static_cast<int64_t>(tile_begin + it) * 128));
+        load_k_tile(sK + s * C::K_BYTES, &tmap_k, &full[s], paged, sPage, it,
+                    kstart + static_cast<int64_t>(tile_begin + it) * 128);
       }
     }
   } else if (warp == 1) {
@@ -221,8 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_items = n_tiles * C::NG;
     // k_scale of this thread's key in the group's next item, fetched one item ahead
     auto key_scale = [&](int item) {
-      const int s = (tile_begin + item / C::NG) * 128 + key_in_tile;
-      return (item < n_items && s < kv) ? __ldg(&p.k_scale[kstart + s]) : 0.f;
+      const int it = item / C::NG;
+      const int s = (tile_begin + it) * 128 + key_in_tile;
+      return (item < n_items && s < kv) ? scale_of_key(p.k_scale, paged, sPage, it, key_in_tile, kstart + s,
+                                                       p.total_keys)
+                                        : 0.f;
     };
     float ks_next = key_scale(g);
     for (int item = g; item < n_items; item += kAccBufs) {
@@ -326,12 +374,14 @@ struct FusedCfg {
   static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // tmem slot (4) + pad (12) | counts [TOK][2] (16) | scan scratch [32] (128) | broadcast [4] (16)
-  static constexpr int OFF_CNT = OFF_MISC + 16;
-  static constexpr int OFF_WARP = OFF_CNT + 16;
+  // tmem slot (4) + pad (12) | exchange slots [8] + per-rank counts [16] (96) | scan scratch [32] (128)
+  // | broadcast [4] (16) | paged caches: pool rows of the chunk's 64-key halves [2 * CAPT / 128]
+  static constexpr int OFF_CNT = (OFF_MISC + 16 + 15) / 16 * 16;   // 16-byte aligned: read as v4 by peers
+  static constexpr int OFF_WARP = OFF_CNT + 96;
   static constexpr int OFF_BC = OFF_WARP + 128;
-  static constexpr int SMEM = OFF_BC + 16 + 1024;
-  static_assert(OFF_K % 1024 == 0 && OFF_S % 16 == 0 && OFF_HIST % 16 == 0, "alignment");
+  static constexpr int OFF_PAGE = OFF_BC + 16;
+  static constexpr int SMEM = OFF_PAGE + 4 * (2 * CAPT / 128) + 1024;
+  static_assert(OFF_K % 1024 == 0 && OFF_S % 16 == 0 && OFF_HIST % 16 == 0 && OFF_CNT % 16 == 0, "alignment");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -455,6 +505,209 @@ __device__ void cluster_radix_topk(const float* __restrict__ sc, int len, int p0
   __syncthreads();           // s_bc / s_warp are reused by the next row
 }
 
+// The row's top k by value bins, the common case.  Scratch (16 KB of shared
+// memory per CTA): [0, 8K) histogram, later the chunk's bitmask of selected
+// boundary positions; [8K, 12K) this CTA's boundary candidates (values,
+// positions); [12K, 16K) every CTA's candidates.  slots[0..5] are read by the
+// other CTAs of the cluster; slots[6] is local.
+//   1. cluster-wide range [lo, hi] of the scores (and whether any is not finite);
+//   2. a 2048-bin histogram over equal-width value bins of [lo, hi] (an fma
+//      of the value, so bins are ordered like the scores), all-reduced over
+//      the cluster: the bin b* holding the k-th largest score;
+//   3. every position above b* is selected; the positions inside b* (tens on
+//      indexer rows) are gathered from all CTAs and ranked exactly (higher
+//      score, then lower position) by every CTA alike;
+//   4. each CTA writes its selected positions, ascending, at its offset.
+// Rows with a non-finite score, a single value, or more than kCandCap
+// positions in b* return false before writing anything (uniformly across the
+// cluster); the caller then runs the radix select.
+constexpr int kCandCap = 512;
+
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+__device__ bool cluster_value_topk(const float* __restrict__ sc, int len, int p0, int k, int32_t* __restrict__ out,
+                                   uint8_t* scratch, uint32_t* slots, uint32_t* s_warp, uint32_t* s_bc, int C,
+                                   uint32_t crank) {
+  constexpr int NT = kThreads;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t FULL = 0xffffffffu;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(scratch);
+  float* own_v = reinterpret_cast<float*>(scratch + 8192);
+  int32_t* own_p = reinterpret_cast<int32_t*>(scratch + 10240);
+  float* all_v = reinterpret_cast<float*>(scratch + 12288);
+  int32_t* all_p = reinterpret_cast<int32_t*>(scratch + 14336);
+
+  // ---- 1. range ----
+  if (tid == 0) {
+    slots[0] = 0u;            // max key
+    slots[1] = 0xFFFFFFFFu;   // min key
+    slots[2] = 0u;            // any non-finite
+    slots[4] = 0u;            // positions above b*
+    slots[5] = 0u;            // boundary candidates
+  }
+  __syncthreads();
+  {
+    uint32_t kmax = 0u, kmin = 0xFFFFFFFFu, bad = 0u;
+    for (int e = tid; e < len; e += NT) {
+      const float x = sc[e];
+      if (!(fabsf(x) <= 3.402823466e38f)) {
+        bad = 1u;
+      } else {
+        const uint32_t key = order_key(x);
+        kmax = max(kmax, key);
+        kmin = min(kmin, key);
+      }
+    }
+    kmax = __reduce_max_sync(FULL, kmax);
+    kmin = __reduce_min_sync(FULL, kmin);
+    bad = __reduce_or_sync(FULL, bad);
+    if (lane == 0) {
+      atomicMax(&slots[0], kmax);
+      atomicMin(&slots[1], kmin);
+      atomicOr(&slots[2], bad);
+    }
+  }
+  __syncthreads();
+  cluster_sync();                          // (1) every CTA's range is visible
+  uint32_t gmax = 0u, gmin = 0xFFFFFFFFu, gbad = 0u;
+  for (int r = 0; r < C; ++r) {
+    const uint4 v = ld_shared_cluster_v4(mapa_shared(smem_u32(slots), static_cast<uint32_t>(r)));
+    gmax = max(gmax, v.x);
+    gmin = min(gmin, v.y);
+    gbad |= v.z;
+  }
+  if (gbad != 0u || gmax <= gmin) return false;   // uniform: every CTA read the same slots
+  const float lo = key_to_float(gmin), hi = key_to_float(gmax);
+  const float scale = static_cast<float>(kRadixBins) / (hi - lo);
+  if (!(scale <= 3.0e38f)) return false;           // a range too narrow for float bins
+  const float off = 8388608.0f - lo * scale;
+  auto bin_of = [&](float x) -> int {
+    const int bb = static_cast<int>(__float_as_uint(__fmaf_rn(x, scale, off))) - 0x4B000000;
+    return min(max(bb, 0), kRadixBins - 1);
+  };
+
+  // ---- 2. histogram of value bins, cluster-wide ----
+  for (int j = tid; j < kRadixBins; j += NT) hist[j] = 0u;
+  __syncthreads();
+  for (int e = tid; e < len; e += NT) atomicAdd(&hist[bin_of(sc[e])], 1u);
+  __syncthreads();
+  cluster_sync();                          // (2) every CTA's histogram is complete
+  uint32_t v[4] = {0u, 0u, 0u, 0u};        // bins 2047 - (4 tid + j), summed over the cluster
+  if (tid < kRadixBins / 4) {
+    const uint32_t a = smem_u32(hist + kRadixBins - 4 - 4 * tid);
+    for (int r = 0; r < C; ++r) {
+      const uint4 h = ld_shared_cluster_v4(mapa_shared(a, static_cast<uint32_t>(r)));
+      v[0] += h.w;
+      v[1] += h.z;
+      v[2] += h.y;
+      v[3] += h.x;
+    }
+  }
+  uint32_t total;
+  uint32_t above = block_excl_scan<NT>(v[0] + v[1] + v[2] + v[3], s_warp, total);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (above < static_cast<uint32_t>(k) && above + v[j] >= static_cast<uint32_t>(k)) {
+      s_bc[0] = static_cast<uint32_t>(kRadixBins - 1 - (4 * tid + j));
+      s_bc[1] = above;
+      s_bc[2] = v[j];
+    }
+    above += v[j];
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(s_bc[0]);
+  const uint32_t above_all = s_bc[1];
+  if (s_bc[2] > static_cast<uint32_t>(kCandCap)) {
+    cluster_sync();                        // nobody reads our histogram any more
+    return false;
+  }
+  const uint32_t rem = static_cast<uint32_t>(k) - above_all;
+
+  // ---- 3. above b*: counted; inside b*: candidates ----
+  {
+    uint32_t n_above = 0;
+    for (int e = tid; e < len; e += NT) {
+      const float x = sc[e];
+      const int bb = bin_of(x);
+      n_above += bb > bstar;
+      if (bb == bstar) {
+        const uint32_t slot = atomicAdd(&slots[5], 1u);    // < kCandCap: the cluster's b* count is
+        own_v[slot] = x;
+        own_p[slot] = p0 + e;
+      }
+    }
+    n_above = __reduce_add_sync(FULL, n_above);
+    if (lane == 0 && n_above) atomicAdd(&slots[4], n_above);
+  }
+  __syncthreads();
+  cluster_sync();                          // (3) every CTA's candidates and counts are visible
+  // gather all candidates (in rank order of their CTAs) and every CTA's count above b*
+  uint32_t n_all = 0, my_base = 0, my_n = 0, base_above = 0;
+  {
+    for (int r = 0; r < C; ++r) {
+      const uint2 c = ld_shared_cluster_v2(mapa_shared(smem_u32(slots + 4), static_cast<uint32_t>(r)));
+      const uint32_t src_v = mapa_shared(smem_u32(own_v), static_cast<uint32_t>(r));
+      const uint32_t src_p = mapa_shared(smem_u32(own_p), static_cast<uint32_t>(r));
+      for (uint32_t i = tid; i < c.y; i += NT) {
+        uint32_t vb, pb;
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(vb) : "r"(src_v + 4 * i) : "memory");
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(pb) : "r"(src_p + 4 * i) : "memory");
+        all_v[n_all + i] = __uint_as_float(vb);
+        all_p[n_all + i] = static_cast<int32_t>(pb);
+      }
+      if (static_cast<uint32_t>(r) == crank) {
+        my_base = n_all;
+        my_n = c.y;
+      }
+      if (static_cast<uint32_t>(r) < crank) base_above += c.x;
+      n_all += c.y;
+    }
+  }
+  __syncthreads();
+  // ---- 4. rank the candidates (every CTA ranks the same list the same way);
+  // this CTA's output offset and the bitmap of its selected candidates ----
+  uint32_t* bits = hist;                   // the histogram is dead: every CTA read it before (3)
+  for (int j = tid; j < (len + 31) / 32; j += NT) bits[j] = 0u;
+  if (tid == 0) slots[6] = 0u;             // selected candidates of lower ranks (local only)
+  __syncthreads();
+  for (uint32_t i = tid; i < n_all; i += NT) {
+    const float x = all_v[i];
+    const int pos = all_p[i];
+    uint32_t rk = 0;
+    for (uint32_t j = 0; j < n_all; ++j) {
+      const float y = all_v[j];
+      rk += (y > x) || (y == x && all_p[j] < pos);
+    }
+    if (rk < rem) {
+      if (i < my_base) {
+        atomicAdd(&slots[6], 1u);          // candidates come grouped by rank, lower ranks first
+      } else if (i < my_base + my_n) {
+        const int e = pos - p0;
+        atomicOr(&bits[e >> 5], 1u << (e & 31));
+      }
+    }
+  }
+  __syncthreads();
+  // ---- 5. ordered write: each thread a contiguous run (odd length) ----
+  const uint32_t base = base_above + slots[6];
+  const int seg = ((len + NT - 1) / NT) | 1;
+  const int e0 = min(tid * seg, len), e1 = min(e0 + seg, len);
+  auto chosen = [&](int e) {
+    const int bb = bin_of(sc[e]);
+    return bb > bstar || (bb == bstar && ((bits[e >> 5] >> (e & 31)) & 1u));
+  };
+  uint32_t n_sel = 0;
+  for (int e = e0; e < e1; ++e) n_sel += chosen(e);
+  uint32_t tot;
+  uint32_t o = base + block_excl_scan<NT>(n_sel, s_warp, tot);
+  for (int e = e0; e < e1; ++e)
+    if (chosen(e)) out[o++] = p0 + e;
+  __syncthreads();
+  return true;
+}
+
 template <int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_topk_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -475,8 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kv = __ldg(&p.kv_len[b]);
   const int first = qblock * TOK;
   if (first >= q_len) return;
-  const int64_t kstart = __ldg(&p.kv_start[b]);
-  if (q_len > kv || kv > fp.max_kv_len || kstart < 0 || kstart + kv > p.total_keys) {
+  const int64_t kstart = seq_start(p.pt, p.kv_start, b);
+  if (q_len > kv || kv > fp.max_kv_len || !seq_rows_ok(p.pt, kstart, kv, p.total_keys)) {
     if (threadIdx.x == 0 && crank == 0) report_error(p.err, kDevErrBounds, 151, b);
     return;
   }
@@ -496,6 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = sm + C::OFF_K;
   float* sS = reinterpret_cast<float*>(sm + C::OFF_S);
   uint32_t* hist = reinterpret_cast<uint32_t*>(sm + C::OFF_HIST);
+  uint8_t* scratch = sm + C::OFF_HIST;      // the selection's 16 KB (histograms or candidates)
   float* sW = reinterpret_cast<float*>(sm + C::OFF_W);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
   uint64_t* full = bars;
@@ -504,12 +758,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = q_full + 1;
   uint64_t* acc_empty = q_full + 1 + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(sm + C::OFF_CNT);
+  uint32_t* slots = reinterpret_cast<uint32_t*>(sm + C::OFF_CNT);
   uint32_t* s_warp = reinterpret_cast<uint32_t*>(sm + C::OFF_WARP);
   uint32_t* s_bc = reinterpret_cast<uint32_t*>(sm + C::OFF_BC);
+  int32_t* sPage = reinterpret_cast<int32_t*>(sm + C::OFF_PAGE);
+  const bool paged = p.pt.table != nullptr;
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
+
+  if (paged) stage_half_tile_rows(p.pt, b, kv, tile_begin, n_tiles, p.total_keys, sPage, p.err);
 
   for (int i = threadIdx.x; i < TOK * 64; i += kThreads) {
     const int tk = i >> 6;
@@ -555,8 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(&full[s], C::K_BYTES);
-        tma_load_2d(sK + s * C::K_BYTES, &tmap_k, &full[s], 0,
-                    static_cast<int32_t>(kstart + static_cast<int64_t>(tile_begin + it) * 128));
+        load_k_tile(sK + s * C::K_BYTES, &tmap_k, &full[s], paged, sPage, it,
+                    kstart + static_cast<int64_t>(tile_begin + it) * 128);
       }
     }
   } else if (warp == 1) {
@@ -596,7 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = (quarter * 32u) << 16;
     auto key_scale = [&](int it) {
       const int s = (tile_begin + it) * 128 + key_in_tile;
-      return (it < n_tiles && s < kv) ? __ldg(&p.k_scale[kstart + s]) : 0.f;
+      return (it < n_tiles && s < kv)
+                 ? scale_of_key(p.k_scale, paged, sPage, it, key_in_tile, kstart + s, p.total_keys)
+                 : 0.f;
     };
     float ks_next = key_scale(g);
     for (int it = g; it < n_tiles; it += kAccBufs) {
@@ -661,7 +921,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       continue;
     }
     const int len = min(max(n - p0, 0), n_tiles * 128);
-    cluster_radix_topk(sS + tk * C::CAPT, len, p0, k, out, hist, cnt + 2 * tk, s_warp, s_bc, ncl, crank);
+    const float* sc = sS + tk * C::CAPT;
+    if (!cluster_value_topk(sc, len, p0, k, out, scratch, slots, s_warp, s_bc, ncl, crank))
+      cluster_radix_topk(sc, len, p0, k, out, hist, slots + 6, s_warp, s_bc, ncl, crank);
+    cluster_sync();          // every CTA is done reading this row's slots and candidates
   }
   cluster_sync();            // no CTA leaves while a peer may still read its shared memory
 }
@@ -698,9 +961,12 @@ template <int TOK>
 cudaError_t launch_tok(dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const IndexerParams& p,
                        cudaStream_t stream) {
   using C = IdxCfg<TOK>;
-  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const size_t smem = C::SMEM + (p.pt.table != nullptr ? 8 * static_cast<size_t>(p.tiles_per_chunk) : 0);
+  if (smem > 232448) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  indexer_kernel<TOK><<<grid, kThreads, C::SMEM, stream>>>(tq, tk, p);
+  indexer_kernel<TOK><<<grid, kThreads, smem, stream>>>(tq, tk, p);
   return cudaGetLastError();
 }
 
@@ -731,46 +997,39 @@ int indexer_box_rows_q(int tok) {
   }
 }
 
-// Largest cluster the fused kernel of `tok` tokens can run on this device:
-// 16 (a non-portable size) when the occupancy query finds room for one such
-// cluster, else the portable 8.  Queried once per device.
-static int fused_cluster_cap(int tok) {
-  static std::atomic<int> cache[64][2];
+// Clusters of `c` CTAs of the fused kernel (`tok` tokens) that can be
+// resident at once on this device (cudaOccupancyMaxActiveClusters; 0 when the
+// size cannot run).  Queried once per device and size.
+static int fused_active_clusters(int tok, int c) {
+  static std::atomic<int> cache[64][2][5];   // sizes 1, 2, 4, 8, 16
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  std::atomic<int>& slot = cache[dev][tok == 2 ? 1 : 0];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return c <= 8 ? 1 : 0;
+  const int li = c == 1 ? 0 : c == 2 ? 1 : c == 4 ? 2 : c == 8 ? 3 : 4;
+  std::atomic<int>& slot = cache[dev][tok == 2 ? 1 : 0][li];
   int v = slot.load(std::memory_order_relaxed);
-  if (v != 0) return v;
-  v = 8;
+  if (v != 0) return v - 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(16, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(c), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(c);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (tok == 2) {
-    auto kern = indexer_topk_kernel<2>;
-    cfg.dynamicSmemBytes = FusedCfg<2>::SMEM;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<2>::SMEM) == cudaSuccess &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-        cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1)
-      v = 16;
-  } else {
-    auto kern = indexer_topk_kernel<1>;
-    cfg.dynamicSmemBytes = FusedCfg<1>::SMEM;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FusedCfg<1>::SMEM) == cudaSuccess &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-        cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1)
-      v = 16;
-  }
+  auto query = [&](auto kern, int smem) {
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return;
+    if (c > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) return;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+  };
+  if (tok == 2) query(indexer_topk_kernel<2>, FusedCfg<2>::SMEM);
+  else query(indexer_topk_kernel<1>, FusedCfg<1>::SMEM);
   cudaGetLastError();   // a refused query leaves no sticky error behind
-  slot.store(v, std::memory_order_relaxed);
-  return v;
+  slot.store(n + 1, std::memory_order_relaxed);
+  return n;
 }
 
 int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len) {
@@ -778,13 +1037,15 @@ int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len) {
   const int tiles = (max_kv_len + 127) / 128;
   constexpr int cap_tiles = FusedCfg<1>::CAPT / 128;   // the same per token for both group sizes
   static_assert(FusedCfg<1>::CAPT == FusedCfg<2>::CAPT, "one chunk capacity");
-  const int cmax = fused_cluster_cap(max_q_per_seq);
-  // enough CTAs for the row to fit (memory) and, while the grid stays within
-  // one wave, more of them for bandwidth (each CTA streams its chunk of keys)
+  // enough CTAs for the row to fit in shared memory ...
   int c = 1;
-  while (c <= cmax && (tiles + c - 1) / c > cap_tiles) c *= 2;
-  if (c > cmax) return 0;
-  while (2 * c <= cmax && static_cast<int64_t>(num_seqs) * 2 * c <= sm_count() && (tiles + 2 * c - 1) / (2 * c) >= 8)
+  while (c <= 16 && (tiles + c - 1) / c > cap_tiles) c *= 2;
+  if (c > 16) return 0;
+  if (c > 8 && fused_active_clusters(max_q_per_seq, c) < 1) return 0;
+  // ... and, while every cluster stays resident at once and each CTA keeps
+  // >= 8 key tiles, more of them for bandwidth (each CTA streams its chunk)
+  while (2 * c <= 16 && static_cast<int64_t>(num_seqs) * 2 * c <= sm_count() &&
+         (tiles + 2 * c - 1) / (2 * c) >= 8 && fused_active_clusters(max_q_per_seq, 2 * c) >= num_seqs)
     c *= 2;
   return c;
 }

@@ -6,10 +6,50 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/dsa.h"
+
 namespace dsa {
 
 // SMs of the current device (queried once per device)
 int sm_count();
+
+// Flat or paged caches.  Flat (table == nullptr): position s of sequence b is
+// row kv_start[b] + s.  Paged: row table[b * stride + s / page] * page +
+// s % page of a pool of num_pages pages.
+struct PageTable {
+  const int32_t* table = nullptr;
+  int32_t page = 0;        // rows per page, a multiple of 64
+  int32_t stride = 0;      // entries per sequence in the table
+  int32_t num_pages = 0;
+};
+
+// Host side, shared by the C ABI translation units: the batch descriptor's
+// argument checks (DSA_OK or the status to return) and its page table.
+dsa_status_t validate_batch(const dsa_batch_t* b);
+PageTable batch_pages(const dsa_batch_t* b);
+#ifdef __CUDACC__
+// First cache row of sequence b (flat caches; 0 when paged, where kv_start
+// may be null).
+__device__ __forceinline__ int64_t seq_start(const PageTable& pt, const int64_t* kv_start, int b) {
+  return pt.table == nullptr ? __ldg(&kv_start[b]) : 0;
+}
+
+// Every position 0 .. kv-1 of the sequence has a cache row: inside the flat
+// cache, or inside the sequence's block-table row.
+__device__ __forceinline__ bool seq_rows_ok(const PageTable& pt, int64_t kstart, int kv, int64_t total_keys) {
+  if (pt.table == nullptr) return kstart >= 0 && kstart + kv <= total_keys;
+  return static_cast<int64_t>(kv) <= static_cast<int64_t>(pt.stride) * pt.page;
+}
+
+// Cache row of position s (>= 0) of sequence b, or -1 when the page id in the
+// block table is outside the pool.
+__device__ __forceinline__ int64_t cache_row(const PageTable& pt, int b, int64_t kstart, int s) {
+  if (pt.table == nullptr) return kstart + s;
+  const int pg = __ldg(&pt.table[static_cast<int64_t>(b) * pt.stride + s / pt.page]);
+  if (pg < 0 || pg >= pt.num_pages) return -1;
+  return static_cast<int64_t>(pg) * pt.page + s % pt.page;
+}
+#endif
 
 // clock64 cycles one bounded device wait may take before it records
 // DSA_ERR_DEVICE_TIMEOUT: DSA_WAIT_BUDGET_CYCLES if set (> 0), else ~1 s
@@ -30,6 +70,7 @@ struct IndexerParams {
   int32_t num_qblocks;      // gridDim.y
   uint32_t* err;
   long long budget;         // clock64 cycles per bounded wait
+  PageTable pt;             // paged: the k tiles load as two 64-row boxes from their pages
 };
 
 // tokens per CTA: 1, 2, 4 or 8
@@ -94,6 +135,7 @@ struct MlaParams {
   const int32_t* idx = nullptr;       // [total_q, k_sel]
   int64_t total_keys = 0;
   int32_t total_q = 0;                // rows of q / out / lse / idx
+  PageTable pt;
   int32_t k_sel = 0;
   int32_t n_heads = 0;
   float scale_log2 = 0.f;             // sm_scale * log2(e)
@@ -140,8 +182,8 @@ cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t str
 cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales, cudaStream_t stream);
 // new tokens' keys (quantised) and latent rows into the flat caches
 cudaError_t launch_cache_write(int num_seqs, int max_q_per_seq, int total_q, int64_t total_keys,
-                               const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start, const void* k,
-                               const void* latent, void* k_cache, float* k_scale, void* latent_cache, uint32_t* err,
-                               cudaStream_t stream);
+                               const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start,
+                               const PageTable& pt, const void* k, const void* latent, void* k_cache, float* k_scale,
+                               void* latent_cache, uint32_t* err, cudaStream_t stream);
 
 }  // namespace dsa

@@ -71,6 +71,7 @@ struct CacheWriteParams {
   const int32_t* cu_q;
   const int32_t* kv_len;
   const int64_t* kv_start;
+  PageTable pt;
   const uint2* k;          // bf16 [total_q, 128]
   const uint4* latent;     // bf16 [total_q, 576]
   uint32_t* k_cache;       // e4m3 [total_keys, 128]
@@ -90,13 +91,17 @@ __global__ void __launch_bounds__(kWarps * 32) cache_write_kernel(const CacheWri
   const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
   if (tok >= q_len) return;
   const int kv = __ldg(&p.kv_len[b]);
-  const int64_t ks = __ldg(&p.kv_start[b]);
-  if (q0 < 0 || q0 + q_len > p.total_q || q_len > kv || ks < 0 || ks + kv > p.total_keys) {
+  const int64_t ks = seq_start(p.pt, p.kv_start, b);
+  if (q0 < 0 || q0 + q_len > p.total_q || q_len > kv || !seq_rows_ok(p.pt, ks, kv, p.total_keys)) {
     if (lane == 0) report_error(p.err, kDevErrBounds, 401, b);
     return;
   }
   const int64_t src = q0 + tok;
-  const int64_t dst = ks + (kv - q_len + tok);   // the token's position t = kv - q_len + tok
+  const int64_t dst = cache_row(p.pt, b, ks, kv - q_len + tok);   // the token's position t = kv - q_len + tok
+  if (dst < 0) {                                                  // a page id outside the pool
+    if (lane == 0) report_error(p.err, kDevErrBounds, 402, b);
+    return;
+  }
   float s;
   const uint32_t c = quant_lane(__ldg(p.k + src * 32 + lane), s);
   p.k_cache[dst * 32 + lane] = c;
@@ -117,13 +122,14 @@ cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float
 }
 
 cudaError_t launch_cache_write(int num_seqs, int max_q_per_seq, int total_q, int64_t total_keys,
-                               const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start, const void* k,
-                               const void* latent, void* k_cache, float* k_scale, void* latent_cache, uint32_t* err,
-                               cudaStream_t stream) {
+                               const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start,
+                               const PageTable& pt, const void* k, const void* latent, void* k_cache, float* k_scale,
+                               void* latent_cache, uint32_t* err, cudaStream_t stream) {
   CacheWriteParams p;
   p.cu_q = cu_q;
   p.kv_len = kv_len;
   p.kv_start = kv_start;
+  p.pt = pt;
   p.k = static_cast<const uint2*>(k);
   p.latent = static_cast<const uint4*>(latent);
   p.k_cache = static_cast<uint32_t*>(k_cache);

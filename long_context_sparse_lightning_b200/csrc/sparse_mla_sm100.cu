@@ -207,8 +207,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     return;
   }
   const int kv = __ldg(&p.kv_len[b]);
-  const int64_t kstart = __ldg(&p.kv_start[b]);
-  if (q_len > kv || kstart < 0 || kstart + kv > p.total_keys) {
+  const int64_t kstart = seq_start(p.pt, p.kv_start, b);
+  if (q_len > kv || !seq_rows_ok(p.pt, kstart, kv, p.total_keys)) {
     if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 301, b);
     // The row attends to nothing: out = 0 and lse = -inf (split partials:
     // lse = -inf, which the merge turns into the same), so no stale partial
@@ -247,6 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   // ---- this split's selected positions: loads first (one memory latency,
   // overlapping the set-up below) ----
   const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
+  // (positions are checked against kv_len and mapped to cache rows below)
   constexpr int PER = (2048 + C::THREADS - 1) / C::THREADS;
   int v[PER];
 #pragma unroll
@@ -290,14 +291,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   }
   __syncthreads();
 
-  // ---- invalid -> -1, per-32 validity bits, the last valid slot ----
+  // ---- each selected position -> its cache row (flat or paged), invalid -> -1,
+  // per-32 validity bits, the last valid slot ----
   int my_last = -1;
   {
 #pragma unroll
     for (int q = 0; q < PER; ++q) {
       const int j = tid + q * C::THREADS;
       if (j < 2048) {
-        const int e = (v[q] < 0 || v[q] >= kv) ? -1 : v[q];
+        int e = (v[q] < 0 || v[q] >= kv) ? -1 : v[q];
+        if (e >= 0) {
+          const int64_t r = cache_row(p.pt, b, kstart, e);
+          if (r < 0) report_error(p.err, kDevErrBounds, 303, b);   // a page id outside the pool: skipped
+          e = static_cast<int>(r);
+        }
         sIdx[j] = e;
         const uint32_t bits = __ballot_sync(0xffffffffu, e >= 0);
         if (lane == 0) sValid[j >> 5] = bits;
@@ -326,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // covers a few whole 128-byte lines.  bf16 sources are converted to fp16 in
     // place by the thread that loaded them.  Two tiles ahead.
     if (n_tiles > 0) {
-      const uint8_t* kvbase = reinterpret_cast<const uint8_t*>(p.kv + kstart * 576);
+      const uint8_t* kvbase = reinterpret_cast<const uint8_t*>(p.kv);   // sIdx holds cache rows
       // this thread's units (the same slots in every tile): unit g = tid + m * PTHREADS
       // of the tile is row j = g / 36, 16-byte unit u = g % 36
       constexpr int UPT = (kTileUnits + C::PTHREADS - 1) / C::PTHREADS;

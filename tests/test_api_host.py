@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert dsa.version() == 100
+    assert dsa.version() == 200
     lib = dsa.library()
     for code in range(7):
         assert lib.dsa_status_string(code).decode()
@@ -171,3 +171,23 @@ def test_quantize_binding_checks_shapes_before_the_call():
     with pytest.raises(ValueError):
         dsa.quantize_fp8(torch.zeros((3, 64), dtype=torch.bfloat16), torch.zeros((3, 64), dtype=torch.uint8),
                          torch.zeros(3, dtype=torch.float32))
+
+
+def test_paged_batch_checks():
+    lib = dsa.library()
+
+    def paged(page, blocks, total_keys=64 * 40, max_kv=1000):
+        c = _host_batch(max_kv=max_kv, total_keys=total_keys)
+        c.kv_start = None                    # ignored (may be null) with a block table
+        c.block_table = 0x2000
+        c.page_size, c.blocks_per_seq = page, blocks
+        return c
+
+    ok = paged(64, 16)
+    assert lib.dsa_workspace_size(dsa.OP_INDEXER, ctypes.byref(ok), 64, 16) == 256
+    for bad in (paged(32, 32), paged(96, 11), paged(64, 15),          # page not a multiple of 64; table too short
+                paged(64, 16, total_keys=64 * 40 + 1)):               # pool not a whole number of pages
+        assert lib.dsa_workspace_size(dsa.OP_INDEXER, ctypes.byref(bad), 64, 16) == 0
+    flat_null = _host_batch()
+    flat_null.kv_start = None                # flat caches need kv_start
+    assert lib.dsa_workspace_size(dsa.OP_INDEXER, ctypes.byref(flat_null), 64, 16) == 0
