@@ -417,6 +417,8 @@ def measure(x, args, dev, pg, world, full, min_region_s=0.0):
     sec = slowest_rank(sum(a.elapsed_time(c) for a, c in ev) / 1e3, pg, dev)
     res = {"steps": steps, "sec": sec, "value": whole_job_rate(world, b.total_q, steps, sec),
            "launches_per_step": dsa.forward_launches(batch, k, H), "clocks": clk.summary()}
+    if getattr(args, "forward_only", False):      # profiling runs: the forward launches and nothing else
+        return res
 
     # ---- per-stage device time (same stream, CUDA events between the launches) ----
     ld = ((b.max_kv_len + 3) // 4) * 4
@@ -552,6 +554,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="measure only --workload (by default a 1-GPU run also measures the other four configs)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="for profiler command lines: only the warm-up and timed forward steps of --workload "
+                         "(no stage timing, end-to-end run, preparation kernels, other configs or CPU baseline)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_setup(args)
@@ -571,7 +576,17 @@ def main():
         pg = td
 
     x = make_inputs(args.workload, seed=rank)
-    r = measure(x, args, dev, pg, world, full=True)
+    r = measure(x, args, dev, pg, world, full=not args.forward_only)
+    if args.forward_only:
+        if pg:
+            pg.barrier()
+            pg.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
+                              "steps": r["steps"], "warmup": args.warmup, "ms_per_step": 1e3 * r["sec"] / r["steps"],
+                              "forward_only": True, "config": config_of(x, args),
+                              "gpu_launches": r["launches_per_step"] * r["steps"], "clocks": r["clocks"]}), flush=True)
+        return 0
     extra = {}
     if world == 1 and not args.no_extra_workloads:
         for name in EXTRA_WORKLOADS:

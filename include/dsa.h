@@ -122,6 +122,7 @@ typedef struct {
  * this includes the [total_q, ld] fp32 score matrix, ld = max_kv_len rounded
  * up to 4 -- except for decode batches (at most 2 query tokens per sequence,
  * rows the fused kernel's clusters hold), whose scores never leave the chip.
+ * (dsa_forward: only where it takes the fused kernel, see dsa_indexer_topk).
  * For DSA_OP_TOPK (and the unfused forward) rows longer than 32768 positions
  * with k_sel a multiple of 4 add 8 * k_sel bytes per row and 32768-position
  * segment: the candidates of the two-phase selection. */
@@ -150,7 +151,8 @@ DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int
 /* Indexer scores and top-k in one call: `idx` as dsa_topk returns it for the
  * scores dsa_indexer_scores computes, bit for bit.  For decode batches (at
  * most 2 query tokens per sequence, rows of up to 16 x 16384 positions) one
- * fused kernel does both ("DeepSeek V3.2 稀疏注意力", what happens in prefill
+ * fused kernel always does both (dsa_forward takes it only where it is the
+ * faster path: one query token per sequence, enough sequences to fill the GPU) ("DeepSeek V3.2 稀疏注意力", what happens in prefill
  * and decode: score tile by tile, keep local candidates, merge, and hand the
  * selection to sparse MLA without writing the score matrix to HBM): a
  * cluster of CTAs per sequence scores one contiguous key chunk per CTA into
@@ -161,6 +163,34 @@ DSA_API dsa_status_t dsa_topk(const dsa_batch_t* batch, const float* scores, int
 DSA_API dsa_status_t dsa_indexer_topk(const dsa_batch_t* batch, const void* q_fp8, const float* q_scale,
                                       const float* w, const void* k_fp8, const float* k_scale, int32_t k_sel,
                                       int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Key-sharded selection ("DeepSeek V3.2 稀疏注意力", top-k section: with the
+ * keys split across devices, select a local top k per shard, then merge the
+ * shards' candidates).  Each of a row's top k lies in the top k of its own
+ * shard, so the merge equals a selection over the whole row.
+ *
+ * dsa_topk_candidates: dsa_topk over one shard's scores (the batch describes
+ * the shard: kv_len = the shard's positions, which start at global position
+ * pos_offset[b] of sequence b), writing each selected position as a global one
+ * and its score:
+ *   cand_pos [total_q, k_sel] int32 out: pos_offset[b] + local position,
+ *            ascending, -1 padding (pos_offset may be NULL: offsets 0)
+ *   cand_val [total_q, k_sel] fp32 out: the scores; padding gets a NaN whose
+ *            order key is below every score.
+ *   ws as for dsa_topk. */
+DSA_API dsa_status_t dsa_topk_candidates(const dsa_batch_t* batch, const float* scores, int64_t ld_scores,
+                                         int32_t k_sel, const int32_t* pos_offset, int32_t* cand_pos,
+                                         float* cand_val, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* dsa_topk_merge: per row, the k_sel highest-scoring of n_src candidate lists
+ * of k_sel entries each (the shards' dsa_topk_candidates outputs, gathered in
+ * shard order, shards covering ascending position ranges):
+ *   cand_pos [n_rows, n_src, k_sel] int32, cand_val [n_rows, n_src, k_sel] fp32
+ *   idx      [n_rows, k_sel] int32 out: positions ascending, -1 padding.
+ * Ties as in dsa_topk (the lower position wins).  n_src * k_sel <= 32768 and a
+ * multiple of 4 (else DSA_ERR_UNSUPPORTED).  No workspace. */
+DSA_API dsa_status_t dsa_topk_merge(int32_t n_rows, int32_t n_src, int32_t k_sel, const int32_t* cand_pos,
+                                    const float* cand_val, int32_t* idx, dsa_stream_t stream);
 
 /* Sparse MLA (MQA mode).
  *   q    [total_q, n_heads, 576] bf16        kv [total_keys, 576] bf16 latent cache

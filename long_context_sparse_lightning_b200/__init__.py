@@ -41,6 +41,8 @@ EXPORTS = [
     "dsa_indexer_scores",
     "dsa_topk",
     "dsa_indexer_topk",
+    "dsa_topk_candidates",
+    "dsa_topk_merge",
     "dsa_sparse_mla",
     "dsa_forward",
     "dsa_sparse_mla_no_alloc",
@@ -96,6 +98,10 @@ def _lib():
         lib.dsa_topk.restype = ctypes.c_int
         lib.dsa_indexer_topk.argtypes = [BP, P, P, P, P, P, I32, P, P, SZ, P]
         lib.dsa_indexer_topk.restype = ctypes.c_int
+        lib.dsa_topk_candidates.argtypes = [BP, P, I64, I32, P, P, P, P, SZ, P]
+        lib.dsa_topk_candidates.restype = ctypes.c_int
+        lib.dsa_topk_merge.argtypes = [I32, I32, I32, P, P, P, P]
+        lib.dsa_topk_merge.restype = ctypes.c_int
         lib.dsa_sparse_mla.argtypes = [BP, P, I32, P, P, I32, F, P, P, P, SZ, P]
         lib.dsa_sparse_mla.restype = ctypes.c_int
         lib.dsa_forward.argtypes = [BP, P, P, P, P, P, I32, P, I32, P, F, P, P, P, P, SZ, P]
@@ -222,6 +228,21 @@ def indexer_topk(batch: Batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel: int, id
     """Indexer scores and top-k in one call (fused on chip for decode batches)."""
     _check(_lib().dsa_indexer_topk(batch.ref, _ptr(q_fp8), _ptr(q_scale), _ptr(w), _ptr(k_fp8), _ptr(k_scale), k_sel,
                                    _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
+
+
+def topk_candidates(batch: Batch, scores, k_sel: int, cand_pos, cand_val, ws, pos_offset=None, stream=None):
+    """One key shard's top k as global positions (+ pos_offset per sequence) and their scores."""
+    _check(_lib().dsa_topk_candidates(batch.ref, _ptr(scores), scores.shape[-1], k_sel, _ptr(pos_offset),
+                                      _ptr(cand_pos), _ptr(cand_val), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_topk_candidates")
+
+
+def topk_merge(cand_pos, cand_val, k_sel: int, idx, stream=None):
+    """Top k per row over [n_rows, n_src, k_sel] candidate lists (shards in position order)."""
+    if cand_pos.dim() != 3 or cand_pos.shape != cand_val.shape or cand_pos.shape[2] != k_sel:
+        raise ValueError("topk_merge: cand_pos / cand_val [n_rows, n_src, k_sel]")
+    _check(_lib().dsa_topk_merge(int(cand_pos.shape[0]), int(cand_pos.shape[1]), k_sel, _ptr(cand_pos),
+                                 _ptr(cand_val), _ptr(idx), _stream(stream)), "dsa_topk_merge")
 
 
 def sparse_mla(batch: Batch, q, kv, idx, k_sel: int, sm_scale: float, out, lse, ws, stream=None):

@@ -178,6 +178,7 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
   p.err = err;
   p.budget = wait_budget();
   p.pt = page_table(b);
+  p.skip_arrival = dsa::test_skip_arrival();
   const dim3 grid((tiles + tpc - 1) / tpc, qblocks, b->num_seqs);
   return dsa::launch_indexer(tok, grid, tq, tk, p, stream) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -185,6 +186,11 @@ dsa_status_t run_indexer(const dsa_batch_t* b, const void* q_fp8, const float* q
 // The fused decode indexer + top-k applies (CTAs per cluster), or 0.
 int fused_cluster(const dsa_batch_t* b) {
   return dsa::indexer_topk_cluster(b->max_q_per_seq, b->num_seqs, b->max_kv_len);
+}
+
+// dsa_forward takes the fused kernel (it applies and is the faster path).
+bool forward_fused(const dsa_batch_t* b) {
+  return dsa::indexer_topk_preferred(b->max_q_per_seq, b->num_seqs, fused_cluster(b));
 }
 
 dsa_status_t run_indexer_topk(const dsa_batch_t* b, const void* q_fp8, const float* q_scale, const float* w,
@@ -323,6 +329,13 @@ dsa_status_t check_mla_args(const void* q, int n_heads, const void* kv, int k_se
 
 namespace dsa {
 dsa_status_t validate_batch(const dsa_batch_t* b) { return check_batch(b); }
+
+int test_skip_arrival() {
+  const char* s = std::getenv("DSA_TEST_SKIP_ARRIVAL");
+  if (s == nullptr || *s == '\0') return -1;
+  const long v = std::atol(s);
+  return v >= 0 && v < (1L << 30) ? static_cast<int>(v) : -1;
+}
 PageTable batch_pages(const dsa_batch_t* b) { return page_table(b); }
 
 long long wait_budget() {
@@ -364,7 +377,7 @@ size_t dsa_workspace_size(dsa_op_t op, const dsa_batch_t* batch, int32_t k_sel, 
       return kHeaderBytes + scores_bytes(batch) + topk_ws_bytes(batch, k_sel);
     case DSA_OP_FORWARD: {
       if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
-      if (fused_cluster(batch) > 0) return kHeaderBytes + mla_ws_bytes(batch, k_sel);
+      if (forward_fused(batch)) return kHeaderBytes + mla_ws_bytes(batch, k_sel);
       // the top-k candidates and the MLA buffers are used one after the other
       return kHeaderBytes + scores_bytes(batch) + std::max(mla_ws_bytes(batch, k_sel), topk_ws_bytes(batch, k_sel));
     }
@@ -429,7 +442,7 @@ dsa_status_t dsa_forward(const dsa_batch_t* batch, const void* q_fp8, const floa
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
   uint8_t* part;
-  if (fused_cluster(batch) > 0) {          // decode: scores stay on chip
+  if (forward_fused(batch)) {              // decode: scores stay on chip
     part = base + kHeaderBytes;
     if ((s = run_indexer_topk(batch, q_fp8, q_scale, w, k_fp8, k_scale, k_sel, idx, err, st)) != DSA_OK) return s;
   } else {
@@ -464,12 +477,57 @@ dsa_status_t dsa_indexer_topk(const dsa_batch_t* batch, const void* q_fp8, const
   return run_topk(batch, scores, ld, k_sel, idx, base + kHeaderBytes + scores_bytes(batch), err, st);
 }
 
+dsa_status_t dsa_topk_candidates(const dsa_batch_t* batch, const float* scores, int64_t ld_scores, int32_t k_sel,
+                                 const int32_t* pos_offset, int32_t* cand_pos, float* cand_val, void* ws,
+                                 size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status_t s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if (scores == nullptr || cand_pos == nullptr || cand_val == nullptr || !aligned16(scores) ||
+      ld_scores < batch->max_kv_len || (ld_scores & 3) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (pos_offset != nullptr && (reinterpret_cast<uintptr_t>(pos_offset) & 3u) != 0) return DSA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes + topk_ws_bytes(batch, k_sel))) != DSA_OK) return s;
+  if (batch->total_q == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((s = run_topk(batch, scores, ld_scores, k_sel, cand_pos, static_cast<uint8_t*>(ws) + kHeaderBytes,
+                    static_cast<uint32_t*>(ws), st)) != DSA_OK)
+    return s;
+  dsa::TopkParams p;
+  p.cu_q = batch->cu_q;
+  p.kv_len = batch->kv_len;
+  p.scores = scores;
+  p.ld = ld_scores;
+  p.k_sel = k_sel;
+  p.idx = cand_pos;
+  p.total_q = batch->total_q;
+  p.num_seqs = batch->num_seqs;
+  p.err = static_cast<uint32_t*>(ws);
+  p.budget = wait_budget();
+  return dsa::launch_topk_values(p, pos_offset, cand_val, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t dsa_topk_merge(int32_t n_rows, int32_t n_src, int32_t k_sel, const int32_t* cand_pos,
+                            const float* cand_val, int32_t* idx, dsa_stream_t stream) {
+  if (n_rows < 0 || n_src < 1 || cand_pos == nullptr || cand_val == nullptr || idx == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(cand_pos) || !aligned16(cand_val)) return DSA_ERR_INVALID_ARG;
+  if (k_sel < 1 || k_sel > DSA_MAX_K_SEL) return DSA_ERR_UNSUPPORTED;
+  const int64_t m = static_cast<int64_t>(n_src) * k_sel;
+  if (m > 32768 || (m & 3) != 0) return DSA_ERR_UNSUPPORTED;
+  if (n_rows == 0) return DSA_OK;
+  return dsa::launch_topk_merge_sources(n_rows, n_src, k_sel, cand_pos, cand_val, idx,
+                                        reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DSA_OK
+             : DSA_ERR_CUDA;
+}
+
 int32_t dsa_forward_launches(const dsa_batch_t* batch, int32_t k_sel, int32_t n_heads) {
   if (check_batch(batch) != DSA_OK) return 0;
   if (k_sel < 1 || k_sel > DSA_MAX_K_SEL || n_heads < 1 || n_heads > 128) return 0;
   if (batch->total_q == 0) return 0;
   int32_t n = 1;                                                             // indexer (fused: + top-k)
-  if (fused_cluster(batch) == 0) n += dsa::topk_segments(batch->max_kv_len, k_sel, batch->total_q).segs > 0 ? 2 : 1;
+  if (!forward_fused(batch)) n += dsa::topk_segments(batch->max_kv_len, k_sel, batch->total_q).segs > 0 ? 2 : 1;
   if (mla_copy(batch, k_sel)) n += 1;                                        // fp16 latent copy
   n += 1;                                                                    // sparse MLA
   if (mla_split(batch, k_sel).nsplit > 1) n += 1;                            // merge

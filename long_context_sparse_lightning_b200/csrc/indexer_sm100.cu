@@ -52,7 +52,7 @@ struct IdxCfg {
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_W = OFF_K + STAGES * K_BYTES;
   static constexpr int OFF_BAR = OFF_W + TOK * 64 * 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs;
+  static constexpr int NUM_BARS = 2 * STAGES + 1 + 2 * kAccBufs + 1;   // + the MMA warp's drain barrier
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_PAGE = OFF_MISC + 16;      // paged caches: pool row of each 64-key half tile
   static constexpr int SMEM = OFF_PAGE + 1024;        // + slack for 1024-byte alignment (+ 8 B per tile when paged)
@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars + 2 * C::STAGES;
   uint64_t* acc_full = q_full + 1;               // [kAccBufs]
   uint64_t* acc_empty = q_full + 1 + kAccBufs;    // [kAccBufs]
+  uint64_t* mma_done = acc_empty + kAccBufs;       // every MMA of this CTA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
   int32_t* sPage = reinterpret_cast<int32_t*>(sm + C::OFF_PAGE);
 
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);   // one arrival per epilogue warp of the group
     }
+    mbar_init(mma_done, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -198,6 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // failure-path tests: this CTA withholds one accumulator release
+  const int skip_item =
+      (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) ? p.skip_arrival : -1;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer --
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int piece = 0; piece < (TOK * 64) / C::BOXQ; ++piece) {
         tma_load_2d(sQ + piece * C::BOXQ * 128, &tmap_q, q_full, 0, row0 * 64 + piece * C::BOXQ);
       }
+      int issued = 0;
       for (int it = 0; it < n_tiles; ++it) {
         const int s = it % C::STAGES;
         const uint32_t ph = (it / C::STAGES) & 1;
@@ -219,7 +225,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], C::K_BYTES);
         load_k_tile(sK + s * C::K_BYTES, &tmap_k, &full[s], paged, sPage, it,
                     kstart + static_cast<int64_t>(tile_begin + it) * 128);
+        issued = it + 1;
       }
+      // No copy may still be writing shared memory when the CTA leaves: wait
+      // for the last load of every stage (already complete on the normal
+      // path, where the MMA warp consumed them) and for the q tile.
+      for (int it = max(0, issued - C::STAGES); it < issued; ++it) {
+        if (!mbar_wait(&full[it % C::STAGES], (it / C::STAGES) & 1, p.budget))
+          report_error(p.err, kDevErrTimeout, 111, it);
+      }
+      if (!mbar_wait(q_full, 0, p.budget)) report_error(p.err, kDevErrTimeout, 112, 0);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer --
@@ -255,6 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&empty[s]);
       }
+      // every MMA (and commit) of this CTA has completed before anyone frees
+      // TMEM or leaves, whether the loop ran to the end or stopped on a timeout
+      umma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0, p.budget)) report_error(p.err, kDevErrTimeout, 123, 0);
     }
   } else {
     // --------------------------------------------------- epilogue --
@@ -321,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[g]);
+      if (lane == 0 && item != skip_item) mbar_arrive(&acc_empty[g]);
     }
   }
 
@@ -1048,6 +1067,17 @@ int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len) {
          (tiles + 2 * c - 1) / (2 * c) >= 8 && fused_active_clusters(max_q_per_seq, 2 * c) >= num_seqs)
     c *= 2;
   return c;
+}
+
+bool indexer_topk_preferred(int max_q_per_seq, int num_seqs, int cluster) {
+  // The fused kernel pays its cluster-wide selection once per token (~15 us
+  // of passes and cluster barriers) and streams the keys with only
+  // num_seqs x cluster CTAs; it beats the indexer + top-k pair (measured) for
+  // one-token groups spread over at least ~2/3 of the SMs (64 x 16K-32K:
+  // 70 vs 77 us; 16 x 32K: 40 vs 54 us), not for two-token groups on few
+  // sequences (8 x 2 at 128K: 99 vs 81 us).
+  return cluster > 0 && max_q_per_seq == 1 &&
+         static_cast<int64_t>(num_seqs) * cluster * 3 >= static_cast<int64_t>(sm_count()) * 2;
 }
 
 cudaError_t launch_indexer_topk(int tok, int cluster, dim3 grid, const CUtensorMap& tmap_q,

@@ -71,7 +71,14 @@ struct IndexerParams {
   uint32_t* err;
   long long budget;         // clock64 cycles per bounded wait
   PageTable pt;             // paged: the k tiles load as two 64-row boxes from their pages
+  int32_t skip_arrival = -1;  // failure-path tests only: CTA (0,0,0) skips its epilogue's
+                              // release of this accumulator item (see test_skip_arrival)
 };
+
+// Item whose accumulator release CTA (0,0,0) of the indexer skips, so that a
+// bounded wait runs out: DSA_TEST_SKIP_ARRIVAL, read per call; -1 (unset) in
+// normal use.  For tests of the device error path only.
+int test_skip_arrival();
 
 // tokens per CTA: 1, 2, 4 or 8
 int indexer_tokens_per_cta(int max_q_per_seq);
@@ -93,6 +100,9 @@ struct IndexerTopkParams {
 // CTAs per cluster for this batch, 0 when the fused kernel does not apply
 // (more than 2 tokens per sequence, or a row too long for 16 CTAs).
 int indexer_topk_cluster(int max_q_per_seq, int num_seqs, int max_kv_len);
+// Whether dsa_forward should take the fused kernel (it is not always faster
+// than the indexer + top-k pair; dsa_indexer_topk takes it whenever it applies).
+bool indexer_topk_preferred(int max_q_per_seq, int num_seqs, int cluster);
 cudaError_t launch_indexer_topk(int tok, int cluster, dim3 grid, const CUtensorMap& tmap_q,
                                 const CUtensorMap& tmap_k, const IndexerTopkParams& p, cudaStream_t stream);
 
@@ -124,6 +134,12 @@ struct TopkSegments {
 };
 TopkSegments topk_segments(int max_kv_len, int k_sel, int total_q);
 cudaError_t launch_topk(int max_kv_len, const TopkParams& p, cudaStream_t stream);
+// p.idx (local positions, as launch_topk wrote them) -> global positions
+// (+ pos_offset[sequence], may be null) in place, and their scores into vals
+cudaError_t launch_topk_values(const TopkParams& p, const int32_t* pos_offset, float* vals, cudaStream_t stream);
+// top k of n_src candidate lists of k entries per row (n_src * k <= 32768, a multiple of 4)
+cudaError_t launch_topk_merge_sources(int n_rows, int n_src, int k, const int32_t* cand_pos, const float* cand_val,
+                                      int32_t* idx, cudaStream_t stream);
 
 // ------------------------------------------------------------- sparse MLA --
 struct MlaParams {

@@ -767,6 +767,114 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p
   for (int j = tid; j < k; j += BLOCK) out[j] = __ldcg(&cpos[__ldcg(&out[j])]);   // candidate -> position
 }
 
+// ---- key-sharded selection: a shard's candidates, and their merge ----
+// "DeepSeek V3.2 稀疏注意力", top-k section: with the keys split across
+// devices, each shard selects its local top k and the shards' candidates are
+// merged into the global top k.  Each of a row's top k is in the top k of its
+// own shard, so the merge equals a selection over the whole row.
+
+// In place: idx (a shard's selected local positions, ascending, -1 padded)
+// becomes global positions (+ the sequence's offset) and val their scores
+// (-NaN for padding: its order key is below every score, -inf included).
+__global__ void __launch_bounds__(256) topk_values_kernel(const TopkParams p, const int32_t* __restrict__ pos_offset,
+                                                          float* __restrict__ vals) {
+  const int r = blockIdx.x;
+  int n = 0;
+  if (!row_info(p, r, n)) return;                     // the selection reported it
+  int lo = 0, hi = p.num_seqs;                        // the row's sequence
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(&p.cu_q[mid]) <= r) lo = mid;
+    else hi = mid;
+  }
+  const int off = pos_offset != nullptr ? __ldg(&pos_offset[lo]) : 0;
+  int32_t* row = p.idx + static_cast<int64_t>(r) * p.k_sel;
+  float* v = vals + static_cast<int64_t>(r) * p.k_sel;
+  const float* sc = p.scores + static_cast<int64_t>(r) * p.ld;
+  for (int j = threadIdx.x; j < p.k_sel; j += blockDim.x) {
+    const int q = row[j];
+    v[j] = q >= 0 ? __ldg(&sc[q]) : __int_as_float(0xFFFFFFFF);
+    row[j] = q >= 0 ? q + off : -1;
+  }
+}
+
+// One CTA per row: the top k of n_src candidate lists of k entries (global
+// positions ascending across the lists, -1 = none).  Candidate index order is
+// position order, so the lower-position tie rule carries over.
+template <int BLOCK, int EPT>
+__global__ void __launch_bounds__(BLOCK, 1) topk_merge_sources_kernel(const int32_t* __restrict__ cand_pos,
+                                                                      const float* __restrict__ cand_val, int m,
+                                                                      int k, int32_t* __restrict__ idx) {
+  __shared__ TopkShared<BLOCK, BLOCK * EPT / 32> sh;
+  const int tid = threadIdx.x, r = blockIdx.x;
+  const int32_t* cp = cand_pos + static_cast<int64_t>(r) * m;
+  const float* cv = cand_val + static_cast<int64_t>(r) * m;
+  int32_t* out = idx + static_cast<int64_t>(r) * k;
+  // valid candidates, in order (each thread a contiguous odd-length run)
+  const int seg = ((m + BLOCK - 1) / BLOCK) | 1;
+  const int e0 = min(tid * seg, m), e1 = min(e0 + seg, m);
+  uint32_t nv = 0;
+  for (int e = e0; e < e1; ++e) nv += __ldg(&cp[e]) >= 0;
+  uint32_t total;
+  uint32_t o = block_excl_scan<BLOCK>(nv, sh.s_warp, total);
+  if (total <= static_cast<uint32_t>(k)) {           // every valid candidate, then -1
+    for (int e = e0; e < e1; ++e) {
+      const int q = __ldg(&cp[e]);
+      if (q >= 0) out[o++] = q;
+    }
+    for (int j = static_cast<int>(total) + tid; j < k; j += BLOCK) out[j] = -1;
+    return;
+  }
+  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
+  __syncthreads();
+  const int n_vec = m >> 2;                           // m is a multiple of 4
+  const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
+  const float4* v4 = reinterpret_cast<const float4*>(cv);
+  const int4* p4 = reinterpret_cast<const int4*>(cp);
+  const float NN = __int_as_float(0xFFFFFFFF);        // padding: below every score
+  float x[EPT];
+#pragma unroll
+  for (int v = 0; v < EPT / 4; ++v) {
+    const int vec = v * BLOCK + tid;
+    float4 f = load_padded(v4, vec, n_vec, m, true);
+    if (vec < n_vec) {
+      const int4 q = __ldcg(&p4[vec]);
+      if (q.x < 0) f.x = NN;
+      if (q.y < 0) f.y = NN;
+      if (q.z < 0) f.z = NN;
+      if (q.w < 0) f.w = NN;
+    }
+    x[4 * v + 0] = f.x;
+    x[4 * v + 1] = f.y;
+    x[4 * v + 2] = f.z;
+    x[4 * v + 3] = f.w;
+  }
+  auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
+  if (!select_fast<BLOCK, EPT>(sh, get4, m, n_chunks, k, x[0], out)) {
+    // the register row, read back through a functor that keeps the padding rule
+    struct Masked {
+      const float4* v4;
+      const int4* p4;
+      int n_vec;
+      __device__ float4 operator()(int v) const {
+        const int vec = v * BLOCK + static_cast<int>(threadIdx.x);
+        if (vec >= n_vec) return make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 f = __ldcg(v4 + vec);
+        const int4 q = __ldcg(p4 + vec);
+        const float NN2 = __int_as_float(0xFFFFFFFF);
+        if (q.x < 0) f.x = NN2;
+        if (q.y < 0) f.y = NN2;
+        if (q.z < 0) f.z = NN2;
+        if (q.w < 0) f.w = NN2;
+        return f;
+      }
+    };
+    select_radix<BLOCK>(sh, Masked{v4, p4, n_vec}, m, n_chunks, k, out);
+  }
+  __syncthreads();
+  for (int j = tid; j < k; j += BLOCK) out[j] = __ldcg(&cp[__ldcg(&out[j])]);   // candidate -> position
+}
+
 template <int BLOCK, int EPT, int MIN_CTAS>
 cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
   constexpr size_t smem = reg_smem_bytes<BLOCK, EPT>();
@@ -779,6 +887,21 @@ cudaError_t launch_reg(const TopkParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_topk_values(const TopkParams& p, const int32_t* pos_offset, float* vals, cudaStream_t stream) {
+  if (p.total_q <= 0) return cudaSuccess;
+  topk_values_kernel<<<p.total_q, 256, 0, stream>>>(p, pos_offset, vals);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_merge_sources(int n_rows, int n_src, int k, const int32_t* cand_pos, const float* cand_val,
+                                      int32_t* idx, cudaStream_t stream) {
+  if (n_rows <= 0) return cudaSuccess;
+  const int m = n_src * k;
+  if (m > 1024 * 32 || (m & 3) != 0) return cudaErrorInvalidValue;
+  topk_merge_sources_kernel<1024, 32><<<n_rows, 1024, 0, stream>>>(cand_pos, cand_val, m, k, idx);
+  return cudaGetLastError();
+}
 
 int sm_count() {
   // per-device cache; concurrent first calls store the same value

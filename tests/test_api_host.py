@@ -74,13 +74,13 @@ def test_forward_launch_counts():
     # one long-context sequence of many queries: + the fp16 latent copy
     pre = _host_batch(B=1, total_q=4096, max_q=4096, max_kv=32768, total_keys=32768)
     assert lib.dsa_forward_launches(ctypes.byref(pre), 2048, 128) == 4
-    # a few decode tokens at 128K: the fused indexer + top-k, split selections + merge
+    # a few two-token groups at 128K: two-phase top-k and split selections + merge
     dec = _host_batch(B=8, total_q=16, max_q=2, max_kv=131072, total_keys=8 * 131072)
-    assert lib.dsa_forward_launches(ctypes.byref(dec), 2048, 128) == 3
+    assert lib.dsa_forward_launches(ctypes.byref(dec), 2048, 128) == 5
     assert lib.dsa_forward_launches(ctypes.byref(dec), 4096, 128) == 0      # k_sel too large
-    # three query tokens per sequence: no fused kernel; two-phase top-k at 128K
-    dec3 = _host_batch(B=8, total_q=24, max_q=3, max_kv=131072, total_keys=8 * 131072)
-    assert lib.dsa_forward_launches(ctypes.byref(dec3), 2048, 128) == 5
+    # 64 one-token decode rows: the fused indexer + top-k, then the sparse MLA
+    dec1 = _host_batch(B=64, total_q=64, max_q=1, max_kv=32768, total_keys=64 * 32768)
+    assert lib.dsa_forward_launches(ctypes.byref(dec1), 2048, 128) == 2
 
 
 def test_fused_decode_workspace_holds_no_scores():

@@ -70,11 +70,13 @@ def test_fused_equal_scores_split_ties_by_position():
 
 
 def test_forward_on_decode_uses_no_score_matrix():
-    # the forward's workspace of a decode batch has no room for the scores, and
+    # one-token decode rows over enough sequences to fill the GPU: the forward
+    # takes the fused kernel (its workspace has no room for the scores), and
     # its selection equals the two-kernel one
-    x = make_inputs(custom_workload("fused_fwd", [9000, 7000, 12000], [1, 1, 1], k_sel=2048, n_heads=128), seed=33)
+    x = make_inputs(custom_workload("fused_fwd", [3000 + 17 * i for i in range(64)], [1] * 64, k_sel=2048,
+                                    n_heads=16), seed=33)
     g = GpuRun(x)
-    ws_fwd = dsa.workspace_size(dsa.OP_FORWARD, g.batch, 2048, 128)
-    assert ws_fwd == dsa.workspace_size(dsa.OP_SPARSE_MLA, g.batch, 2048, 128)
+    ws_fwd = dsa.workspace_size(dsa.OP_FORWARD, g.batch, 2048, 16)
+    assert ws_fwd == dsa.workspace_size(dsa.OP_SPARSE_MLA, g.batch, 2048, 16)
     idx_f, _, _ = g.forward(2048)
     assert torch.equal(idx_f, g.topk(g.scores(), 2048))
