@@ -285,6 +285,27 @@ DSA_API dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* batch, const voi
 DSA_API dsa_status_t dsa_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales,
                                       dsa_stream_t stream);
 
+/* dsa_indexer_prep: the whole input chain of the indexer's q or k vectors
+ * ("详解DSA", indexer code: rotary embedding on the first 64 dims of each
+ * 128-dim vector, then rotate_activation, then act_quant; "DeepSeek V3.2
+ * 稀疏注意力": the indexer takes the non-interleaved RoPE layout).  Readings
+ * (the pages define neither function): dims i and i + 32 (i < 32) rotate by
+ * (rope_cos, rope_sin)[pos][i], out_i = x_i c - x_{i+32} s and out_{i+32} =
+ * x_{i+32} c + x_i s in fp32 without fused multiply-adds, stored as bf16;
+ * rotate_activation is the normalised Walsh-Hadamard transform over the 128
+ * dims (Sylvester order, butterfly stages 1, 2, ..., 64 in fp32, times
+ * fp32(128^-0.5)), stored as bf16; then the quantiser above.
+ *   x        [n_vec, 128] bf16; vector v belongs to position pos[v / vecs_per_pos]
+ *            (vecs_per_pos = 64 for q, the token's head vectors; 1 for k)
+ *   pos      [n_vec / vecs_per_pos] int32 positions, 0 <= pos < n_pos
+ *   rope_cos, rope_sin  [n_pos, 32] fp32 tables (the caller's frequencies)
+ *   codes    [n_vec, 128] e4m3 out;  scales [n_vec] fp32 out
+ *   ws       >= 256 bytes (device error word): a position outside the table is
+ *            DSA_ERR_DEVICE_BOUNDS, its vector written as codes 0, scale 1. */
+DSA_API dsa_status_t dsa_indexer_prep(const void* x, int64_t n_vec, int32_t vecs_per_pos, const int32_t* pos,
+                                      const float* rope_cos, const float* rope_sin, int32_t n_pos, void* codes,
+                                      float* scales, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* dsa_cache_write: the keys and latent rows of the batch's new tokens into the
  * flat caches.  Query row r (sequence b, position t, see "Ragged batches")
  * writes cache row kv_start[b] + t:

@@ -51,6 +51,7 @@ EXPORTS = [
     "dsa_version",
     "dsa_forward_launches",
     "dsa_quantize_fp8",
+    "dsa_indexer_prep",
     "dsa_cache_write",
 ]
 
@@ -118,6 +119,8 @@ def _lib():
         lib.dsa_forward_launches.restype = I32
         lib.dsa_quantize_fp8.argtypes = [P, I64, P, P, P]
         lib.dsa_quantize_fp8.restype = ctypes.c_int
+        lib.dsa_indexer_prep.argtypes = [P, I64, I32, P, P, P, I32, P, P, P, SZ, P]
+        lib.dsa_indexer_prep.restype = ctypes.c_int
         lib.dsa_cache_write.argtypes = [BP, P, P, P, P, P, P, SZ, P]
         lib.dsa_cache_write.restype = ctypes.c_int
         _LIB = lib
@@ -266,6 +269,19 @@ def quantize_fp8(x, codes, scales, stream=None):
         raise ValueError("quantize_fp8: x bf16 [..., 128], codes uint8 of the same size, scales fp32 [...]")
     n_vec = x.numel() // INDEX_DIM
     _check(_lib().dsa_quantize_fp8(_ptr(x), n_vec, _ptr(codes), _ptr(scales), _stream(stream)), "dsa_quantize_fp8")
+
+
+def indexer_prep(x, pos, rope_cos, rope_sin, codes, scales, ws, vecs_per_pos: int, stream=None):
+    """Non-interleaved RoPE on dims 0..63, normalised Walsh-Hadamard, per-128 FP8: x bf16 [..., 128]."""
+    if x.dtype != torch.bfloat16 or x.shape[-1] != INDEX_DIM or codes.dtype != torch.uint8 \
+            or codes.numel() != x.numel() or scales.dtype != torch.float32 or scales.numel() * INDEX_DIM != x.numel() \
+            or pos.dtype != torch.int32 or rope_cos.dtype != torch.float32 or rope_sin.shape != rope_cos.shape \
+            or rope_cos.shape[-1] != 32:
+        raise ValueError("indexer_prep: x bf16 [..., 128], pos int32, rope tables fp32 [n_pos, 32]")
+    n_vec = x.numel() // INDEX_DIM
+    _check(_lib().dsa_indexer_prep(_ptr(x), n_vec, int(vecs_per_pos), _ptr(pos), _ptr(rope_cos), _ptr(rope_sin),
+                                   int(rope_cos.shape[0]), _ptr(codes), _ptr(scales), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "dsa_indexer_prep")
 
 
 def cache_write(batch: Batch, k, latent, k_cache, k_scale, latent_cache, ws, stream=None):

@@ -544,6 +544,25 @@ dsa_status_t dsa_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* 
              : DSA_ERR_CUDA;
 }
 
+dsa_status_t dsa_indexer_prep(const void* x, int64_t n_vec, int32_t vecs_per_pos, const int32_t* pos,
+                              const float* rope_cos, const float* rope_sin, int32_t n_pos, void* codes, float* scales,
+                              void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (n_vec < 0 || vecs_per_pos < 1 || n_pos < 1 || x == nullptr || pos == nullptr || rope_cos == nullptr ||
+      rope_sin == nullptr || codes == nullptr || scales == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(rope_cos) || !aligned16(rope_sin) ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u) != 0 || n_vec % vecs_per_pos != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (n_vec >= (int64_t(1) << 40)) return DSA_ERR_UNSUPPORTED;
+  dsa_status_t s;
+  if ((s = check_ws(ws, ws_bytes, kHeaderBytes)) != DSA_OK) return s;
+  if (n_vec == 0) return DSA_OK;
+  return dsa::launch_indexer_prep(x, n_vec, vecs_per_pos, pos, rope_cos, rope_sin, n_pos, codes, scales,
+                                  static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DSA_OK
+             : DSA_ERR_CUDA;
+}
+
 dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* k, const void* latent, void* k_cache,
                              float* k_scale, void* latent_cache, void* ws, size_t ws_bytes, dsa_stream_t stream) {
   dsa_status_t s = check_batch(batch);

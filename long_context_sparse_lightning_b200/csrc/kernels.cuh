@@ -196,6 +196,10 @@ cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t str
 // ------------------------------------------------------------------- prep --
 // per-128 FP8 quantiser: x bf16 [n_vec, 128] -> codes e4m3 [n_vec, 128], scales [n_vec]
 cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float* scales, cudaStream_t stream);
+// non-interleaved RoPE on dims 0..63 -> normalised Walsh-Hadamard -> per-128 FP8
+cudaError_t launch_indexer_prep(const void* x, int64_t n_vec, int vecs_per_pos, const int32_t* pos,
+                                const float* rope_cos, const float* rope_sin, int n_pos, void* codes, float* scales,
+                                uint32_t* err, cudaStream_t stream);
 // new tokens' keys (quantised) and latent rows into the flat caches
 cudaError_t launch_cache_write(int num_seqs, int max_q_per_seq, int total_q, int64_t total_keys,
                                const int32_t* cu_q, const int32_t* kv_len, const int64_t* kv_start,

@@ -67,6 +67,85 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// The indexer's input chain ("详解DSA", indexer code: the first 64 dims of each
+// q head vector / key get rotary position embedding, then rotate_activation,
+// then act_quant; "DeepSeek V3.2 稀疏注意力": the indexer wants the
+// non-interleaved RoPE layout), fused per 128-element vector, one warp each:
+//   RoPE   dims i and i + 32 (i < 32) rotate by the position's (cos_i, sin_i):
+//          out_i = x_i c - x_{i+32} s, out_{i+32} = x_{i+32} c + x_i s (fp32
+//          products and sums, no fused multiply-add), stored as bf16;
+//   rotate the normalised Walsh-Hadamard transform over the 128 dims
+//          (Sylvester order, butterfly stages h = 1 .. 64 in fp32, then
+//          x fp32(128^-0.5)), stored as bf16;
+//   act_quant as quant_lane.
+// Lane l holds dims 4l .. 4l+3: the RoPE partner of lane l < 8 is lane l + 8,
+// the Hadamard partner at stride h >= 4 is lane l ^ (h / 4).
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h));
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+    indexer_prep_kernel(const uint2* __restrict__ x, int64_t n_vec, int vecs_per_pos, const int32_t* __restrict__ pos,
+                        const float* __restrict__ rope_cos, const float* __restrict__ rope_sin, int n_pos,
+                        uint32_t* __restrict__ codes, float* __restrict__ scales, uint32_t* err) {
+  const uint32_t FULL = 0xffffffffu;
+  const int lane = static_cast<int>(threadIdx.x & 31u);
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  const int64_t n_warps = static_cast<int64_t>(gridDim.x) * kWarps;
+  for (int64_t v = warp; v < n_vec; v += n_warps) {
+    const int p = __ldg(&pos[v / vecs_per_pos]);
+    if (p < 0 || p >= n_pos) {               // warp-uniform: no table row to read
+      if (lane == 0) {
+        report_error(err, kDevErrBounds, 501, static_cast<uint32_t>(v));
+        scales[v] = 1.f;
+      }
+      codes[v * 32 + lane] = 0u;
+      continue;
+    }
+    const uint2 raw = __ldcs(x + v * 32 + lane);
+    float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+    // ---- RoPE on dims 0..63 (lanes 0..15) ----
+    float g[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) g[j] = __shfl_xor_sync(FULL, f[j], 8);
+    if (lane < 16) {
+      const int i0 = 4 * (lane & 7);
+      const float4 c = __ldg(reinterpret_cast<const float4*>(rope_cos + static_cast<int64_t>(p) * 32 + i0));
+      const float4 sn = __ldg(reinterpret_cast<const float4*>(rope_sin + static_cast<int64_t>(p) * 32 + i0));
+      const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {sn.x, sn.y, sn.z, sn.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // lane < 8: (x_i, x_{i+32}) = (f, g); lane >= 8: (x_{i+32}, x_i) = (f, g)
+        const float r = lane < 8 ? __fsub_rn(__fmul_rn(f[j], cc[j]), __fmul_rn(g[j], ss[j]))
+                                 : __fadd_rn(__fmul_rn(f[j], cc[j]), __fmul_rn(g[j], ss[j]));
+        f[j] = __uint_as_float(bf16_bits(r) << 16);
+      }
+    }
+    // ---- Walsh-Hadamard: stages 1, 2 inside the lane, 4 .. 64 across lanes ----
+    float a0 = __fadd_rn(f[0], f[1]), a1 = __fsub_rn(f[0], f[1]);
+    float a2 = __fadd_rn(f[2], f[3]), a3 = __fsub_rn(f[2], f[3]);
+    float b[4] = {__fadd_rn(a0, a2), __fadd_rn(a1, a3), __fsub_rn(a0, a2), __fsub_rn(a1, a3)};
+#pragma unroll
+    for (int m = 1; m <= 16; m <<= 1) {
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float o = __shfl_xor_sync(FULL, b[j], m);
+        b[j] = upper ? __fsub_rn(o, b[j]) : __fadd_rn(b[j], o);
+      }
+    }
+    uint2 rot;
+    rot.x = bf16_bits(__fmul_rn(b[0], 0.08838834764831845f)) | (bf16_bits(__fmul_rn(b[1], 0.08838834764831845f)) << 16);
+    rot.y = bf16_bits(__fmul_rn(b[2], 0.08838834764831845f)) | (bf16_bits(__fmul_rn(b[3], 0.08838834764831845f)) << 16);
+    float sc;
+    const uint32_t cd = quant_lane(rot, sc);
+    codes[v * 32 + lane] = cd;
+    if (lane == 0) scales[v] = sc;
+  }
+}
+
 struct CacheWriteParams {
   const int32_t* cu_q;
   const int32_t* kv_len;
@@ -118,6 +197,18 @@ cudaError_t launch_quantize_fp8(const void* x, int64_t n_vec, void* codes, float
   const int grid = static_cast<int>(need < cap ? need : cap);
   quantize_fp8_kernel<<<grid, kWarps * 32, 0, stream>>>(static_cast<const uint2*>(x), n_vec,
                                                         static_cast<uint32_t*>(codes), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer_prep(const void* x, int64_t n_vec, int vecs_per_pos, const int32_t* pos,
+                                const float* rope_cos, const float* rope_sin, int n_pos, void* codes, float* scales,
+                                uint32_t* err, cudaStream_t stream) {
+  const int64_t need = (n_vec + kWarps - 1) / kWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  indexer_prep_kernel<<<grid, kWarps * 32, 0, stream>>>(static_cast<const uint2*>(x), n_vec, vecs_per_pos, pos,
+                                                        rope_cos, rope_sin, n_pos, static_cast<uint32_t*>(codes),
+                                                        scales, err);
   return cudaGetLastError();
 }
 
