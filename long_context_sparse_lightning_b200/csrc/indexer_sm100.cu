@@ -303,40 +303,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int s = (tile_begin + it) * 128 + key_in_tile;
-#pragma unroll 1
-      for (int tk = 0; tk < C::GTOK; ++tk) {
+      // four running sums (heads j mod 4) kept as two f32x2 pairs: each lane
+      // of fma.rn.f32x2 is the fp32 fma of the scalar form, so the sums are
+      // bit-identical to it, in half the FMA instructions.  Heads 0-31 then
+      // 32-63 of a token, in that order.
+      auto half_sum = [&](const uint32_t (&r)[32], const ulonglong2* w, unsigned long long& a01,
+                          unsigned long long& a23) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const ulonglong2 wv = w[j];
+          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(r[4 * j + 0]), 0.f),
+                                  fmaxf(__uint_as_float(r[4 * j + 1]), 0.f)), a01);
+          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(r[4 * j + 2]), 0.f),
+                                  fmaxf(__uint_as_float(r[4 * j + 3]), 0.f)), a23);
+        }
+      };
+      auto store = [&](int tk, unsigned long long a01, unsigned long long a23) {
         const int tok = grp * C::GTOK + tk;
-        uint32_t ra[32], rb[32];
-        const uint32_t taddr = tmem + lane_addr + static_cast<uint32_t>(g * C::N + tk * 64);
-        tmem_ld32(taddr, ra);
-        tmem_ld32(taddr + 32, rb);
-        tmem_ld_wait();
-        // four running sums (heads j mod 4) kept as two f32x2 pairs: each
-        // lane of fma.rn.f32x2 is the fp32 fma of the scalar form, so the
-        // sums are bit-identical to it, in half the FMA instructions
-        const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(sW + tok * 64);
-        unsigned long long a01 = 0ull, a23 = 0ull;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const ulonglong2 wv = w2[j];
-          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(ra[4 * j + 0]), 0.f),
-                                  fmaxf(__uint_as_float(ra[4 * j + 1]), 0.f)), a01);
-          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(ra[4 * j + 2]), 0.f),
-                                  fmaxf(__uint_as_float(ra[4 * j + 3]), 0.f)), a23);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const ulonglong2 wv = w2[8 + j];
-          a01 = ffma2(wv.x, pack2(fmaxf(__uint_as_float(rb[4 * j + 0]), 0.f),
-                                  fmaxf(__uint_as_float(rb[4 * j + 1]), 0.f)), a01);
-          a23 = ffma2(wv.y, pack2(fmaxf(__uint_as_float(rb[4 * j + 2]), 0.f),
-                                  fmaxf(__uint_as_float(rb[4 * j + 3]), 0.f)), a23);
-        }
         const float2 s01 = unpack2(a01), s23 = unpack2(a23);
         const float acc = (s01.x + s01.y) + (s23.x + s23.y);
-        if (tok < ntok && s <= t_first + tok) {
-          p.scores[static_cast<int64_t>(row0 + tok) * p.ld + s] = acc * ks;
-        }
+        if (tok < ntok && s <= t_first + tok) p.scores[static_cast<int64_t>(row0 + tok) * p.ld + s] = acc * ks;
+      };
+      const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(sW + grp * C::GTOK * 64);
+      const uint32_t taddr = tmem + lane_addr + static_cast<uint32_t>(g * C::N);
+      uint32_t ra[32], rb[32];
+      tmem_ld32(taddr, ra);
+      tmem_ld32(taddr + 32, rb);
+      tmem_ld_wait();
+      unsigned long long a01 = 0ull, a23 = 0ull;
+      half_sum(ra, w2, a01, a23);
+      // a second token: its first half is loaded while the first token's
+      // second half is summed
+      if constexpr (C::GTOK == 2) tmem_ld32(taddr + 64, ra);
+      half_sum(rb, w2 + 8, a01, a23);
+      store(0, a01, a23);
+      if constexpr (C::GTOK == 2) {
+        tmem_ld32(taddr + 96, rb);
+        tmem_ld_wait();
+        a01 = 0ull;
+        a23 = 0ull;
+        half_sum(ra, w2 + 16, a01, a23);
+        half_sum(rb, w2 + 24, a01, a23);
+        store(1, a01, a23);
       }
       tc_fence_before();
       __syncwarp();

@@ -682,7 +682,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       }
       const float refA = m_runA == NEG_INF ? 0.f : m_runA;
       const float refB = m_runB == NEG_INF ? 0.f : m_runB;
-      // next tile's partial scores: wait for the TMEM load, pack, ship
+      // next tile's partial scores: wait for the TMEM load, ship
       if (more) {
         load_s_finish();
         if (!send(i + 1, snext)) {
