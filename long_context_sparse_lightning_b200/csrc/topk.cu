@@ -47,7 +47,7 @@ struct TopkShared {
   float cand_v[kCandCap];
   int32_t cand_p[kCandCap];
   uint8_t cand_sel[kCandCap];
-  uint32_t selbits[CAPW > 0 ? CAPW : 1];   // verdicts of boundary-bin positions, by position
+  uint32_t selbits[CAPW > 0 ? CAPW : 1];   // the row's selection bitmap, one word per 32 positions
   int32_t out_s[kMaxK];                     // the row's output, compacted before one coalesced store
   uint32_t tab[kSegChunks * NW];
   float s_red[4][32];
@@ -295,9 +295,77 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
       }
     });
   };
-  // register rows fit one segment (EPT / 4 <= kSegChunks): classify once
-  static_assert(EPT / 4 <= kSegChunks, "a register row must fit one segment");
-  const bool one_seg = EPT > 0 || n_chunks <= kSegChunks;
+  // Register rows of BLOCK x 32 positions: one 32-bit word of the selection
+  // bitmap per thread.  Classify writes the bits of the positions above b*
+  // (8 lanes' 4-bit nibbles form one word: no atomics), the ranking adds the
+  // chosen b* positions, and thread t then writes the set bits of word t --
+  // positions 32t .. 32t+31, already ascending -- at its offset from one
+  // block-wide scan.
+  if constexpr (EPT > 0 && CAPW == BLOCK) {
+    for_range<EPT>(0, n_chunks, [&](int v) {
+      const float4 f = get4(v);
+      const float e[4] = {f.x, f.y, f.z, f.w};
+      uint32_t cs = 0, cb = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int b = e[c] >= lo ? bin_of(e[c]) : -1;
+        cs |= static_cast<uint32_t>(b > bstar) << c;
+        cb |= static_cast<uint32_t>(b == bstar) << c;
+      }
+      uint32_t wv = cs << (4 * (lane & 7));
+      wv |= __shfl_xor_sync(FULL, wv, 1);
+      wv |= __shfl_xor_sync(FULL, wv, 2);
+      wv |= __shfl_xor_sync(FULL, wv, 4);
+      if ((lane & 7) == 0) sh.selbits[(v * BLOCK + tid) >> 3] = wv;
+      if (__any_sync(FULL, cb != 0u)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool is = (cb >> c) & 1u;
+          const uint32_t m = __ballot_sync(FULL, is);
+          if (m != 0u) {
+            const int leader = __ffs(m) - 1;
+            uint32_t base = 0;
+            if (lane == leader) base = atomicAdd(&sh.s_ncand, static_cast<uint32_t>(__popc(m)));
+            base = __shfl_sync(FULL, base, leader);
+            const uint32_t slot = base + __popc(m & lanemask_lt());
+            if (is && slot < static_cast<uint32_t>(kCandCap)) {
+              sh.cand_v[slot] = e[c];
+              sh.cand_p[slot] = pos_of(v, c);
+            }
+          }
+        }
+      }
+    });
+    __syncthreads();
+    const uint32_t ncand = min(sh.s_ncand, static_cast<uint32_t>(kCandCap));
+    for (uint32_t i = warp; i < ncand; i += NW) {
+      const float x = sh.cand_v[i];
+      const int pos = sh.cand_p[i];
+      uint32_t rank = 0;
+      for (uint32_t j = lane; j < ncand; j += 32) {
+        const float y = sh.cand_v[j];
+        rank += (y > x) || (y == x && sh.cand_p[j] < pos);
+      }
+      rank = __reduce_add_sync(FULL, rank);
+      if (lane == 0 && rank < rem) atomicOr(&sh.selbits[pos >> 5], 1u << (pos & 31));
+    }
+    __syncthreads();
+    // words of chunks past the row were not written for this row
+    uint32_t w = tid < n_chunks * (BLOCK / 8) ? sh.selbits[tid] : 0u;
+    uint32_t total;
+    uint32_t o = block_excl_scan<BLOCK>(static_cast<uint32_t>(__popc(w)), sh.s_warp, total);
+    while (w != 0u) {
+      const int bit = __ffs(w) - 1;
+      w &= w - 1;
+      if (o < static_cast<uint32_t>(k)) out[o] = 32 * tid + bit;
+      ++o;
+    }
+    return true;
+  }
+  // Rows streamed from memory (register rows returned above): classify and
+  // compact segment by segment, the positions' verdicts kept in registers as
+  // 4-bit flags.
+  const bool one_seg = n_chunks <= kSegChunks;
   uint64_t sel = 0, inb = 0;
   if (one_seg) {
     classify(0, n_chunks, true, sel, inb);
@@ -318,13 +386,7 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
       rank += (y > x) || (y == x && sh.cand_p[j] < pos);
     }
     rank = __reduce_add_sync(FULL, rank);
-    if (lane == 0) {
-      if constexpr (CAPW > 0) {
-        if (rank < rem) atomicOr(&sh.selbits[pos >> 5], 1u << (pos & 31));
-      } else {
-        sh.cand_sel[i] = rank < rem;
-      }
-    }
+    if (lane == 0) sh.cand_sel[i] = rank < rem;
   }
   __syncthreads();
 
@@ -340,12 +402,8 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
       inb &= inb - 1;
       const int pos = ((seg0 + (bit >> 2)) * BLOCK + tid) * 4 + (bit & 3);
       bool chosen = false;
-      if constexpr (CAPW > 0) {
-        chosen = (sh.selbits[pos >> 5] >> (pos & 31)) & 1u;
-      } else {
-        for (uint32_t j = 0; j < ncand; ++j)
-          if (sh.cand_p[j] == pos) chosen = sh.cand_sel[j];
-      }
+      for (uint32_t j = 0; j < ncand; ++j)
+        if (sh.cand_p[j] == pos) chosen = sh.cand_sel[j];
       if (chosen) sel |= uint64_t(1) << bit;
     }
     for_range<EPT>(seg0, seg1, [&](int v) {
@@ -400,9 +458,6 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
     __syncthreads();
   }
   for (int j = tid; j < k; j += BLOCK) out[j] = sh.out_s[j];
-  if constexpr (CAPW > 0) {
-    for (uint32_t i = tid; i < ncand; i += BLOCK) sh.selbits[sh.cand_p[i] >> 5] = 0u;
-  }
   return true;
 }
 
@@ -566,7 +621,6 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
     mbar_init(&sh.bar, 1);
     fence_mbar_init();
   }
-  for (int j = tid; j < CAP / 32; j += BLOCK) sh.selbits[j] = 0u;
   __syncthreads();
 
   auto needs_copy = [&](int r, int& n) { return r < p.total_q && row_info(p, r, n) && n > k && n <= CAP; };
@@ -694,7 +748,6 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_segment_kernel(const TopkParams
     }
     return;
   }
-  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
   __syncthreads();
   const int n_vec = (m + 3) >> 2;          // the row stride is a multiple of 4 and >= n
   const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
@@ -744,7 +797,6 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_kernel(const TopkParams p
     for (int j = tid; j < k; j += BLOCK) out[j] = j < m ? __ldcg(&cpos[j]) : -1;
     return;
   }
-  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
   __syncthreads();
   const int n_vec = (m + 3) >> 2;          // k is a multiple of 4 or the tail lies inside the block
   const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
@@ -825,7 +877,6 @@ __global__ void __launch_bounds__(BLOCK, 1) topk_merge_sources_kernel(const int3
     for (int j = static_cast<int>(total) + tid; j < k; j += BLOCK) out[j] = -1;
     return;
   }
-  for (int j = tid; j < BLOCK * EPT / 32; j += BLOCK) sh.selbits[j] = 0u;
   __syncthreads();
   const int n_vec = m >> 2;                           // m is a multiple of 4
   const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
