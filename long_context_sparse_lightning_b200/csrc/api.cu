@@ -271,6 +271,7 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   p.idx = idx;
   p.total_keys = b->total_keys;
   p.total_q = b->total_q;
+  p.num_seqs = b->num_seqs;
   p.pt = page_table(b);
   p.k_sel = k_sel;
   p.n_heads = n_heads;
@@ -288,19 +289,17 @@ dsa_status_t run_mla(const dsa_batch_t* b, const void* q, int n_heads, const voi
   }
   p.err = err;
   p.budget = wait_budget();
-  const int64_t gx = int64_t(2) * b->max_q_per_seq * sp.nsplit;
-  if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
+  if (static_cast<int64_t>(b->total_q) * sp.nsplit >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   dsa::MlaMaps maps;
-  if (!dsa::make_mla_maps(&maps, q, out, b->total_q, n_heads)) return DSA_ERR_CUDA;
+  if (!dsa::make_mla_maps(&maps, q, b->total_q, n_heads)) return DSA_ERR_CUDA;
   if (mla_copy(b, k_sel)) {
     uint16_t* kv16 = reinterpret_cast<uint16_t*>(part + mla_part_bytes(b, k_sel));
     const int64_t n = b->total_keys * 576;
     if (dsa::launch_latent_to_fp16(static_cast<const uint16_t*>(kv), kv16, n, stream) != cudaSuccess)
       return DSA_ERR_CUDA;
     p.kv = kv16;
-    if (dsa::launch_sparse_mla_fp16(grid, p, maps, stream) != cudaSuccess) return DSA_ERR_CUDA;
-  } else if (dsa::launch_sparse_mla(grid, p, maps, stream) != cudaSuccess) {
+    if (dsa::launch_sparse_mla_fp16(p, maps, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  } else if (dsa::launch_sparse_mla(p, maps, stream) != cudaSuccess) {
     return DSA_ERR_CUDA;
   }
   if (sp.nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, stream) != cudaSuccess) return DSA_ERR_CUDA;
@@ -338,6 +337,13 @@ int test_skip_arrival() {
 }
 PageTable batch_pages(const dsa_batch_t* b) { return page_table(b); }
 
+int mla_pair_cap() {
+  const char* s = std::getenv("DSA_MLA_MAX_PAIRS");
+  if (s == nullptr || *s == '\0') return 0;
+  const long v = std::atol(s);
+  return v > 0 && v < (1L << 20) ? static_cast<int>(v) : 0;
+}
+
 long long wait_budget() {
   const char* s = std::getenv("DSA_WAIT_BUDGET_CYCLES");
   if (s != nullptr) {
@@ -347,12 +353,13 @@ long long wait_budget() {
   return kDefaultBudget;
 }
 
-bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads) {
+bool make_mla_maps(MlaMaps* m, const void* q, int64_t total_q, int n_heads) {
   const uint64_t rows = static_cast<uint64_t>(total_q) * static_cast<uint64_t>(n_heads);
   const uint32_t h = static_cast<uint32_t>(n_heads);
+  const uint32_t rope_rows = h < 64 ? h : 64;   // RoPE rows 0-63 and 64-127 travel in separate ring stages
   return make_tmap_2d(&m->q_lat, q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 576, h, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tmap_2d(&m->q_rope, q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 576, h, 32, CU_TENSOR_MAP_SWIZZLE_64B) &&
-         make_tmap_2d(&m->out, out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 512, h, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+         make_tmap_2d(&m->q_rope, q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, rows, 576, rope_rows, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
 }
 }  // namespace dsa
 

@@ -95,6 +95,7 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   p.idx = idx;
   p.total_keys = b->total_keys;
   p.total_q = b->total_q;
+  p.num_seqs = b->num_seqs;
   p.pt = dsa::batch_pages(b);
   p.k_sel = k_sel;
   p.n_heads = n_heads;
@@ -108,12 +109,10 @@ extern "C" dsa_status_t dsa_sparse_mla_no_alloc(const dsa_batch_t* b, const void
   p.part_lse = nsplit > 1 ? reinterpret_cast<float*>(scratch + kHeader + o_bytes) : nullptr;
   p.err = reinterpret_cast<uint32_t*>(scratch);
   p.budget = dsa::wait_budget();
-  const int64_t gx = int64_t(2) * b->max_q_per_seq * nsplit;
-  if (gx >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(gx), b->num_seqs);
+  if (static_cast<int64_t>(b->total_q) * nsplit >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   dsa::MlaMaps maps;
-  if (!dsa::make_mla_maps(&maps, q, out, b->total_q, n_heads)) return DSA_ERR_CUDA;
-  if (dsa::launch_sparse_mla(grid, p, maps, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!dsa::make_mla_maps(&maps, q, b->total_q, n_heads)) return DSA_ERR_CUDA;
+  if (dsa::launch_sparse_mla(p, maps, st) != cudaSuccess) return DSA_ERR_CUDA;
   if (nsplit > 1 && dsa::launch_mla_combine(b->total_q, p, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }

@@ -54,6 +54,9 @@ __device__ __forceinline__ int64_t cache_row(const PageTable& pt, int b, int64_t
 // clock64 cycles one bounded device wait may take before it records
 // DSA_ERR_DEVICE_TIMEOUT: DSA_WAIT_BUDGET_CYCLES if set (> 0), else ~1 s
 long long wait_budget();
+// Test hook: DSA_MLA_MAX_PAIRS=n caps the sparse MLA's persistent grid at n CTA
+// pairs, so that small batches drive many items through each pair; 0 = no cap.
+int mla_pair_cap();
 
 // ---------------------------------------------------------------- indexer --
 struct IndexerParams {
@@ -151,6 +154,7 @@ struct MlaParams {
   const int32_t* idx = nullptr;       // [total_q, k_sel]
   int64_t total_keys = 0;
   int32_t total_q = 0;                // rows of q / out / lse / idx
+  int32_t num_seqs = 0;               // entries of kv_len; cu_q has num_seqs + 1
   PageTable pt;
   int32_t k_sel = 0;
   int32_t n_heads = 0;
@@ -173,23 +177,24 @@ bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_se
 size_t mla_smem_bytes();
 // TMA descriptors of the sparse MLA kernel (bf16 bits as 16-bit elements):
 //   q_lat  over q viewed as [total_q * H, 576], box [H rows x 64 cols], 128-byte swizzle
-//   q_rope the same tensor, box [H rows x 32 cols], 64-byte swizzle
-//   out    over out viewed as [total_q * H, 512], box [H rows x 64 cols], 128-byte swizzle
+//   q_rope the same tensor, box [min(H, 64) rows x 32 cols], 64-byte swizzle
 struct MlaMaps {
   CUtensorMap q_lat;
   CUtensorMap q_rope;
-  CUtensorMap out;
 };
-// Encodes the three descriptors for q [total_q * n_heads, 576] and out
-// [total_q * n_heads, 512]; false if the driver refuses them.
-bool make_mla_maps(MlaMaps* m, const void* q, void* out, int64_t total_q, int n_heads);
+// Encodes both descriptors for q [total_q * n_heads, 576]; false if the driver
+// refuses them.
+bool make_mla_maps(MlaMaps* m, const void* q, int64_t total_q, int n_heads);
 // p.kv is the bf16 cache: selected rows are gathered with 16-byte loads, Q.C^T
 // runs in bf16 on them, and their value part is then converted to fp16 in
 // shared memory for P.V (no extra buffers).
-cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
+// Both launch a persistent grid: one CTA pair per resident cluster slot (at
+// most total_q * nsplit pairs), each pair walking its share of the (token,
+// split) items.
+cudaError_t launch_sparse_mla(const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
 // p.kv is an fp16 copy of the cache (launch_latent_to_fp16): rows are
 // gathered ready for the MMAs.
-cudaError_t launch_sparse_mla_fp16(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
+cudaError_t launch_sparse_mla_fp16(const MlaParams& p, const MlaMaps& maps, cudaStream_t stream);
 cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream);
 cudaError_t launch_mla_combine(int total_q, const MlaParams& p, cudaStream_t stream);
 

@@ -43,13 +43,21 @@
 // noise costs ~1e-3 mean relative error on the bf16 output; fp16 keeps ~1e-4.
 // The conversion of q and the latent entries is exact in the normal fp16 range.
 //
-// Per token, around the tile loop: the CTA's Q slice arrives by TMA boxes into
-// ring stages 2-3 (converted to fp16 into TMEM by the softmax warps before the
-// producers reuse those stages), and the bf16 output leaves by TMA box stores
-// staged, swizzled, in the idle ring.
+// Persistent pairs: each CTA pair walks a share of the (token, split) items.
+// Per item the ring first carries the CTA's Q slice (two stage-sized TMA jobs,
+// moved to TMEM as fp16 by the softmax warps), then the item's tiles; the
+// producers stage the next item's positions and start its Q slice and first
+// gathers while the current item's last tiles are still in the pipeline, and
+// the next item's first Q.C^T runs during the current item's epilogue.  The
+// bf16 output leaves by 16-byte stores of whole 64-byte runs per head (TMEM
+// read with the .32x32b shape: lane = head).  A pair per token with a TMA
+// store epilogue spent ~17K cycles per token outside the tile loop (prologue,
+// epilogue, the next cluster's launch) against ~95K inside it.
 //
 // Decode shapes split a token's selection over several pairs; each writes a
 // normalised partial output and its log-sum-exp, merged by mla_combine_kernel.
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -76,18 +84,19 @@ constexpr int OFF_KV = 0;
 constexpr int OFF_STG = kStages * KV_STAGE;          // 147456: outgoing partial scores (one tile)
 constexpr int OFF_X = OFF_STG + XBUF;                // 180224: incoming partial scores (one tile)
 constexpr int OFF_IDX = OFF_X + XBUF;                // 212992: int32[2048]
-constexpr int OFF_VALID = OFF_IDX + 2048 * 4;        // 221184: uint32[64] validity bits
-constexpr int OFF_BAR = OFF_VALID + 64 * 4;          // 221440
-constexpr int OFF_MISC = OFF_BAR + 512;
+constexpr int OFF_VALID = OFF_IDX + 2048 * 4;        // 221184: uint32[2][64] validity bits (item parity)
+constexpr int OFF_BAR = OFF_VALID + 2 * 64 * 4;      // 221696
+constexpr int OFF_INV = OFF_BAR + 512;               // 222208: float[2][128] inverse row sums (epilogue parity)
+constexpr int OFF_MISC = OFF_INV + 2 * 128 * 4;      // 223232: TMEM address, ItemMeta[2]
 constexpr int kSmem = OFF_MISC + 64 + 1024;
 
 constexpr int kUnitsPerRow = 36;                     // 16-byte units of a row's 288-dim half
 constexpr int kTileUnits = kTileKeys * kUnitsPerRow; // 2304
-constexpr int kQBox = 16384;                         // one 128-row x 128-byte TMA box of Q or O
+constexpr int kQBox = 16384;                         // one (up to) 128-row x 128-byte TMA box of Q
 
 struct Bars {
-  uint64_t q_tma;           // this CTA's Q slice landed in shared memory (TMA)
-  uint64_t q_full;
+  uint64_t q_full;          // the item's Q slice is in TMEM (8 softmax warps)
+  uint64_t q_free;          // the MMA thread has seen that phase of q_full (one per Q slice)
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t qk_done[kStages];   // bf16 source: Q.C^T of the stage's tile has read it (MMA commit)
@@ -95,7 +104,10 @@ struct Bars {
   uint64_t s_full, s_empty;
   uint64_t x_full[8], x_free[8];   // per softmax warp: peer's partial landed / peer has read ours
   uint64_t p_full, pv_done;
-  uint64_t red;            // all softmax warps have staged the output
+  uint64_t red;            // all softmax warps have published their inverse row sums
+  uint64_t meta_full[2];   // item parity: selected positions staged (producers)
+  uint64_t meta_free[2];   // item parity: the softmax warps are done with the validity bits
+  uint64_t pbar;           // producer warps' own barrier (bounded, unlike bar.sync)
 };
 static_assert(sizeof(Bars) <= 512, "");
 
@@ -114,8 +126,11 @@ struct Cfg {
 };
 static_assert(2 * 128 * Cfg::REG_LOW + 2 * 128 * Cfg::REG_HIGH == Cfg::THREADS * 128, "register split");
 static_assert(Cfg::SOFT0 % 4 == 0, "softmax warps must start a warpgroup");
-static_assert(2048 % Cfg::THREADS == 0, "index staging assumes whole warps per pass");
-static_assert(4 * kQBox + 128 * 64 <= 2 * KV_STAGE, "Q slice must fit ring stages 2-3");
+// Index staging: producer thread t takes slots t + 224 q; the last pass (q = 9)
+// covers slots 2016..2047, i.e. exactly warp 0, so every pass is warp-uniform.
+static_assert(9 * Cfg::PTHREADS + 32 == 2048, "index staging passes");
+// A Q slice takes two ring jobs: latent boxes 0-1 (or 2-3) and RoPE rows 0-63 (64-127).
+static_assert(2 * kQBox + 64 * 64 <= KV_STAGE, "half a Q slice must fit one ring stage");
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   const float lo = __uint_as_float(w << 16);
@@ -179,9 +194,77 @@ __device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
   return KV_ROPE + j * 64 + ((ru ^ ((j >> 1) & 3)) << 4);
 }
 
+// What the producers publish about an item (one per item parity, before
+// meta_full): the other roles read it from shared memory instead of
+// recomputing it with dependent global loads.
+struct ItemMeta {
+  int32_t last;     // last valid slot of the selection, -1: none
+  int32_t row, split, status, has_q;
+};
+static_assert(16 + 2 * sizeof(ItemMeta) <= 64, "item metadata fits the misc area");
+
+// Work item w of a launch: token row w / nsplit of the batch, split w % nsplit.
+// status 0: valid; 301: the sequence's descriptors are out of range (the row
+// attends to nothing: out = 0, lse = -inf); 302: the row lies in no sequence
+// of cu_q (nothing of it is written).
+struct MlaItem {
+  int row, split, b, kv, status;
+  int e_begin, e_count;   // the split's slots of the selection (0 slots: nothing to attend)
+  int64_t kstart;
+  // the item carries a Q slice through the ring: every role decides this the
+  // same way, before the positions are staged
+  __device__ __forceinline__ bool has_q() const { return e_count > 0; }
+};
+
+__device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int w) {
+  MlaItem it;
+  it.row = w / p.nsplit;
+  it.split = w - it.row * p.nsplit;
+  // the row's sequence: the last b with cu_q[b] <= row (empty sequences skipped)
+  int lo = 0, hi = p.num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(&p.cu_q[mid]) <= it.row) {
+      lo = mid;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  it.b = lo;
+  it.kv = 0;
+  it.kstart = 0;
+  it.status = 0;
+  it.e_begin = it.split * p.keys_per_split;
+  it.e_count = 0;
+  const int q0 = __ldg(&p.cu_q[lo]);
+  const int q_len = __ldg(&p.cu_q[lo + 1]) - q0;
+  if (q0 < 0 || it.row < q0 || it.row >= q0 + q_len) {
+    it.status = 302;
+    return it;
+  }
+  it.kv = __ldg(&p.kv_len[lo]);
+  it.kstart = seq_start(p.pt, p.kv_start, lo);
+  if (q_len > it.kv || !seq_rows_ok(p.pt, it.kstart, it.kv, p.total_keys)) {
+    it.status = 301;
+    return it;
+  }
+  it.e_count = max(0, min(p.k_sel, it.e_begin + p.keys_per_split) - it.e_begin);
+  return it;
+}
+
 // FP16_SRC: p.kv is an fp16 copy of the latent cache (rows land ready for the
 // MMAs); otherwise p.kv is the bf16 cache: Q.C^T runs in bf16 and the producers
 // convert the value part in place between Q.C^T and P.V.
+//
+// Persistent: gridDim.x / 2 CTA pairs; pair c takes items c, c + pairs, ...
+// Every role walks the same item sequence and keeps the same counters (ring
+// jobs, tiles, items with a Q slice), so the barrier phases agree across
+// items.  Per item with n > 0 tiles the ring carries two Q jobs (the CTA's Q
+// slice by TMA), then the n tiles.  The producers stage the next item's
+// positions and issue its Q slice and first tiles while the current item's
+// last tiles are still in the MMA / softmax pipeline; the softmax warps move
+// the next Q slice into TMEM before the current item's epilogue, so the next
+// item's first Q.C^T overlaps that epilogue.
 template <bool FP16_SRC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     sparse_mla_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
@@ -189,47 +272,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-
   const int pair = static_cast<int>(blockIdx.x >> 1);
-  const int tok = pair / p.nsplit;
-  const int split = pair % p.nsplit;
-  const int b = blockIdx.y;
-  const int q0 = __ldg(&p.cu_q[b]);
-  const int q_len = __ldg(&p.cu_q[b + 1]) - q0;
-  // Every early exit depends only on launch indices and on device inputs that
-  // do not change during the kernel, so both CTAs of a pair take it together
-  // (a one-sided exit would leave the peer waiting in barrier.cluster).
-  if (tok >= q_len) return;
-  const int row = q0 + tok;
+  const int n_pairs = static_cast<int>(gridDim.x >> 1);
+  const int n_items = p.total_q * p.nsplit;
   const int H = p.n_heads;
-  if (q0 < 0 || row >= p.total_q) {          // inconsistent cu_q: nothing of this row is written
-    if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 302, b);
-    return;
-  }
-  const int kv = __ldg(&p.kv_len[b]);
-  const int64_t kstart = seq_start(p.pt, p.kv_start, b);
-  if (q_len > kv || !seq_rows_ok(p.pt, kstart, kv, p.total_keys)) {
-    if (threadIdx.x == 0 && rank == 0) report_error(p.err, kDevErrBounds, 301, b);
-    // The row attends to nothing: out = 0 and lse = -inf (split partials:
-    // lse = -inf, which the merge turns into the same), so no stale partial
-    // of an earlier call is ever merged into this row.
-    const float NI = __int_as_float(0xff800000);
-    if (p.nsplit == 1) {
-      for (int u = threadIdx.x; u < H * 32; u += blockDim.x) {      // 32 16-byte units of this CTA's half
-        const int h = u >> 5, c = u & 31;
-        *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(row) * H + h) * 512 + rank * 256 + c * 8) =
-            make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (rank == 0 && p.lse != nullptr)
-        for (int h = threadIdx.x; h < H; h += blockDim.x) p.lse[static_cast<int64_t>(row) * H + h] = NI;
-    } else {
-      const int64_t prow = (static_cast<int64_t>(row) * p.nsplit + split) * 128;
-      for (int h = threadIdx.x; h < 128; h += blockDim.x) p.part_lse[prow * 2 + rank * 128 + h] = NI;
-    }
-    return;
-  }
-  const int e_begin = split * p.keys_per_split;
-  const int e_count = max(0, min(p.k_sel, e_begin + p.keys_per_split) - e_begin);
 
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -237,32 +283,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   int32_t* sIdx = reinterpret_cast<int32_t*>(sm + OFF_IDX);
   uint32_t* sValid = reinterpret_cast<uint32_t*>(sm + OFF_VALID);
   Bars* bar = reinterpret_cast<Bars*>(sm + OFF_BAR);
+  float* sInv = reinterpret_cast<float*>(sm + OFF_INV);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  int32_t* s_last = reinterpret_cast<int32_t*>(sm + OFF_MISC + 4);
+  ItemMeta* meta = reinterpret_cast<ItemMeta*>(sm + OFF_MISC + 16);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
   const int tid = threadIdx.x;
 
-  // ---- this split's selected positions: loads first (one memory latency,
-  // overlapping the set-up below) ----
-  const int32_t* idx_row = p.idx + static_cast<int64_t>(row) * p.k_sel + e_begin;
-  // (positions are checked against kv_len and mapped to cache rows below)
-  constexpr int PER = (2048 + C::THREADS - 1) / C::THREADS;
-  int v[PER];
-#pragma unroll
-  for (int q = 0; q < PER; ++q) {
-    const int j = tid + q * C::THREADS;
-    v[q] = (j < 2048 && j < e_count) ? __ldg(&idx_row[j]) : -1;
-  }
-
-  // ---- barriers, then this CTA's Q slice by TMA into ring stages 2-3 (free
-  // until the producers' third tile, which waits for q_full) ----
-  uint8_t* sQ = sKV + 2 * KV_STAGE;
   if (tid == 0) {
-    *s_last = -1;
-    mbar_init(&bar->q_tma, 1);
     mbar_init(&bar->q_full, 8);
+    mbar_init(&bar->q_free, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->kv_full[s], C::NPROD);
       mbar_init(&bar->kv_empty[s], 1);
@@ -277,53 +308,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
     mbar_init(&bar->p_full, 8);
     mbar_init(&bar->pv_done, 1);
-    mbar_init(&bar->red, 256);
+    mbar_init(&bar->red, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar->meta_full[i], 1);
+      mbar_init(&bar->meta_free[i], 8);
+    }
+    mbar_init(&bar->pbar, C::NPROD);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&bar->q_tma, static_cast<uint32_t>(H) * (4 * 128 + 64));
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      tma_load_2d(sQ + c * kQBox, &maps.q_lat, &bar->q_tma, static_cast<int>(rank) * 256 + c * 64, row * H);
-    tma_load_2d(sQ + 4 * kQBox, &maps.q_rope, &bar->q_tma, 512 + static_cast<int>(rank) * 32, row * H);
+    prefetch_tmap(&maps.q_lat);
+    prefetch_tmap(&maps.q_rope);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  __syncthreads();
-
-  // ---- each selected position -> its cache row (flat or paged), invalid -> -1,
-  // per-32 validity bits, the last valid slot ----
-  int my_last = -1;
-  {
-#pragma unroll
-    for (int q = 0; q < PER; ++q) {
-      const int j = tid + q * C::THREADS;
-      if (j < 2048) {
-        int e = (v[q] < 0 || v[q] >= kv) ? -1 : v[q];
-        if (e >= 0) {
-          const int64_t r = cache_row(p.pt, b, kstart, e);
-          if (r < 0) report_error(p.err, kDevErrBounds, 303, b);   // a page id outside the pool: skipped
-          e = static_cast<int>(r);
-        }
-        sIdx[j] = e;
-        const uint32_t bits = __ballot_sync(0xffffffffu, e >= 0);
-        if (lane == 0) sValid[j >> 5] = bits;
-        if (e >= 0) my_last = j;
-      }
-    }
-  }
-  if (my_last >= 0) atomicMax(s_last, my_last);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   // Our barriers are initialised: arrive on the cluster barrier now; each role
   // waits for the peer's arrival only before its first remote access (the
-  // softmax warps' first score exchange) or at its end, so the set-up of
-  // both CTAs overlaps the first gathers and the Q conversion.
+  // softmax warps' first score exchange) or at its end.
   cluster_arrive();
   const uint32_t tmem = *tmem_slot;
-  const int n_ent = *s_last + 1;
-  const int n_tiles = (n_ent + kTileKeys - 1) / kTileKeys;
 
   if (warp < C::NPROD) {
     setmaxnreg_dec<C::REG_LOW>();
@@ -332,45 +338,146 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // consecutive lanes take consecutive units of a row, so one warp request
     // covers a few whole 128-byte lines.  bf16 sources are converted to fp16 in
     // place by the thread that loaded them.
-    if (n_tiles > 0) {
-      const uint8_t* kvbase = reinterpret_cast<const uint8_t*>(p.kv);   // sIdx holds cache rows
-      // this thread's units (the same slots in every tile): unit g = tid + m * PTHREADS
-      // of the tile is row j = g / 36, 16-byte unit u = g % 36
-      constexpr int UPT = (kTileUnits + C::PTHREADS - 1) / C::PTHREADS;
-      uint32_t soff[UPT], goff[UPT], jrow[UPT];
+    const uint8_t* kvbase = reinterpret_cast<const uint8_t*>(p.kv);   // sIdx holds cache rows
+    // this thread's units (the same slots in every tile): unit g = tid + m * PTHREADS
+    // of the tile is row j = g / 36, 16-byte unit u = g % 36
+    constexpr int UPT = (kTileUnits + C::PTHREADS - 1) / C::PTHREADS;
+    uint32_t soff[UPT], goff[UPT], jrow[UPT];
 #pragma unroll
-      for (int m = 0; m < UPT; ++m) {
-        const int g = min(tid + m * C::PTHREADS, kTileUnits - 1);
-        const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
-        soff[m] = tile_unit_offset(j, u);
-        goff[m] = static_cast<uint32_t>(unit_dim(u, rank)) * 2u;
-        jrow[m] = static_cast<uint32_t>(j);
+    for (int m = 0; m < UPT; ++m) {
+      const int g = min(tid + m * C::PTHREADS, kTileUnits - 1);
+      const int j = g / kUnitsPerRow, u = g % kUnitsPerRow;
+      soff[m] = tile_unit_offset(j, u);
+      goff[m] = static_cast<uint32_t>(unit_dim(u, rank)) * 2u;
+      jrow[m] = static_cast<uint32_t>(j);
+    }
+    auto mine = [&](int m) { return m + 1 < UPT || tid + m * C::PTHREADS < kTileUnits; };
+    bool ok = true;
+    uint32_t pb = 0;        // uses of the producer barrier
+    // all producer warps (an mbarrier, so that a warp that gave up on an
+    // earlier wait cannot leave the others blocked for good)
+    auto pbar = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->pbar);
+      const bool r = mbar_wait(&bar->pbar, pb & 1u, p.budget);
+      ++pb;
+      if (!__all_sync(0xffffffffu, r)) {
+        if (lane == 0) report_error(p.err, kDevErrTimeout, 314, static_cast<int>(pb));
+        ok = false;
       }
-      auto mine = [&](int m) { return m + 1 < UPT || tid + m * C::PTHREADS < kTileUnits; };
-      bool ok = true;
-      // the tile's ring slot is free: P.V of the slot's previous tile has read
-      // it, and stages 2-3 no longer hold the Q slice (the softmax warps have
-      // moved it to TMEM)
-      auto slot_free = [&](int tile) {
-        const int st = tile % kStages;
-        bool f = mbar_test(smem_u32(&bar->kv_empty[st]), ((tile / kStages) & 1) ^ 1);
-        if (tile == 2 || tile == 3) f = f && mbar_test(smem_u32(&bar->q_full), 0);
-        return __shfl_sync(0xffffffffu, f, 0);   // lane 0 decides for the warp
-      };
+    };
+    // ring job r: stage r % kStages, its use number r / kStages
+    auto slot_wait = [&](int r) {
+      if (ok && !mbar_wait(&bar->kv_empty[r % kStages], ((r / kStages) & 1) ^ 1, p.budget)) {
+        report_error(p.err, kDevErrTimeout, 311, r);
+        ok = false;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+    };
+    int ring = 0;           // ring jobs issued so far (Q halves and tiles)
+    MlaItem nxt;            // the next item, fetched while the current one's Q slice is in flight
+    if (pair < n_items) nxt = mla_item(p, pair);
+    for (int k = 0; ok; ++k) {
+      const int w = pair + k * n_pairs;
+      if (w >= n_items) break;
+      const MlaItem it = nxt;
+      if (it.status != 0 && tid == 0 && rank == 0) report_error(p.err, kDevErrBounds, it.status, it.b);
+      // this item's positions: loads first (one memory latency)
+      const int32_t* idx_row = p.idx + static_cast<int64_t>(it.row) * p.k_sel + it.e_begin;
+      int v[10];
+#pragma unroll
+      for (int q = 0; q < 10; ++q) {
+        const int j = tid + q * C::PTHREADS;
+        v[q] = (j < 2048 && j < it.e_count) ? __ldg(&idx_row[j]) : -1;
+      }
+      // The CTA's Q slice: two ring jobs by TMA (latent boxes 2h, 2h+1 and RoPE
+      // rows 64h..64h+63), issued before the positions are staged so that it
+      // lands while the previous item's last tiles are still being processed.
+      // Every warp waits for the slot before its arrival.
+      if (it.has_q()) {
+        const int rope_rows = H < 64 ? H : 64;
+        for (int h = 0; ok && h < 2; ++h, ++ring) {
+          slot_wait(ring);
+          if (!ok) break;
+          const int st = ring % kStages;
+          if (lane == 0) {
+            // bf16: close the stage's conversion phase for this job first, so
+            // that the job's kv_full completion implies every warp's v_full arrival
+            if constexpr (!FP16_SRC) mbar_arrive(&bar->v_full[st]);
+            if (warp == 0) {
+              const bool rope = h == 0 || H > 64;
+              uint8_t* dst = sKV + st * KV_STAGE;
+              mbar_arrive_expect_tx(&bar->kv_full[st],
+                                    static_cast<uint32_t>(2 * H * 128 + (rope ? rope_rows * 64 : 0)));
+              tma_load_2d(dst, &maps.q_lat, &bar->kv_full[st], static_cast<int>(rank) * 256 + 128 * h, it.row * H);
+              tma_load_2d(dst + kQBox, &maps.q_lat, &bar->kv_full[st], static_cast<int>(rank) * 256 + 128 * h + 64,
+                          it.row * H);
+              if (rope)
+                tma_load_2d(dst + 2 * kQBox, &maps.q_rope, &bar->kv_full[st], 512 + static_cast<int>(rank) * 32,
+                            it.row * H + 64 * h);
+            } else {
+              mbar_arrive(&bar->kv_full[st]);
+            }
+          }
+        }
+        if (!ok) break;
+      }
+      if (w + n_pairs < n_items) nxt = mla_item(p, w + n_pairs);
+      // The previous item's tiles are issued and landed by every warp (sIdx is
+      // free), and the validity buffer of this item's parity is free once the
+      // softmax warps are done with item k - 2.
+      if (tid == 0) {
+        if (k >= 2 && !mbar_wait(&bar->meta_free[k & 1], ((k >> 1) + 1) & 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 315, k);
+          ok = false;
+        }
+        ItemMeta& m = meta[k & 1];
+        m.last = -1;
+        m.row = it.row;
+        m.split = it.split;
+        m.status = it.status;
+        m.has_q = it.has_q() ? 1 : 0;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      pbar();
+      if (!ok) break;
+      // each selected position -> its cache row (flat or paged), invalid -> -1,
+      // per-32 validity bits, the last valid slot
+      uint32_t* sV = sValid + (k & 1) * 64;
+      int my_last = -1;
+#pragma unroll
+      for (int q = 0; q < 10; ++q) {
+        const int j = tid + q * C::PTHREADS;
+        if (j < 2048) {
+          int e = (v[q] < 0 || v[q] >= it.kv) ? -1 : v[q];
+          if (e >= 0) {
+            const int64_t r = cache_row(p.pt, it.b, it.kstart, e);
+            if (r < 0) report_error(p.err, kDevErrBounds, 303, it.b);   // a page id outside the pool: skipped
+            e = static_cast<int>(r);
+          }
+          sIdx[j] = e;
+          const uint32_t bits = __ballot_sync(0xffffffffu, e >= 0);
+          if (lane == 0) sV[j >> 5] = bits;
+          if (e >= 0) my_last = j;
+        }
+      }
+      if (my_last >= 0) atomicMax(&meta[k & 1].last, my_last);
+      pbar();
+      if (!ok) break;
+      const int n_tiles = (meta[k & 1].last + 1 + kTileKeys - 1) / kTileKeys;
+      if (tid == 0) mbar_arrive(&bar->meta_full[k & 1]);
+      if (n_tiles == 0) continue;
+
+      // the item's tiles: ring jobs r0 .. r0 + n_tiles - 1
+      const int r0 = ring;
+      const int32_t* sI = sIdx;
       auto issue = [&](int tile) {
-        const int st = tile % kStages;
-        if (ok && !mbar_wait(&bar->kv_empty[st], ((tile / kStages) & 1) ^ 1, p.budget)) {
-          report_error(p.err, kDevErrTimeout, 311, tile);
-          ok = false;
-        }
-        if (ok && (tile == 2 || tile == 3) && !mbar_wait(&bar->q_full, 0, p.budget)) {
-          report_error(p.err, kDevErrTimeout, 312, tile);
-          ok = false;
-        }
-        ok = __all_sync(0xffffffffu, ok);
+        const int r = r0 + tile;
+        slot_wait(r);
         if (ok) {
-          const uint32_t base = smem_u32(sKV + st * KV_STAGE);
-          const int32_t* e = sIdx + tile * kTileKeys;
+          const uint32_t base = smem_u32(sKV + (r % kStages) * KV_STAGE);
+          const int32_t* e = sI + tile * kTileKeys;
 #pragma unroll
           for (int m = 0; m < UPT; ++m) {
             if (mine(m)) {
@@ -384,33 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       auto land = [&](int tile) {
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->kv_full[tile % kStages]);
-      };
-      // bf16 source: Q.C^T reads the tile as bf16 (exact products, like fp16);
-      // once it has, the value part (units 0..31) becomes fp16 in place for
-      // P.V, off the path from the gather to the scores
-      auto convert = [&](int tile) {
-        if constexpr (!FP16_SRC) {
-          const int st = tile % kStages;
-          if (ok && !mbar_wait(&bar->qk_done[st], (tile / kStages) & 1, p.budget)) {
-            report_error(p.err, kDevErrTimeout, 313, tile);
-            ok = false;
-          }
-          ok = __all_sync(0xffffffffu, ok);
-          if (ok) {
-            uint8_t* base = sKV + st * KV_STAGE;
-#pragma unroll
-            for (int m = 0; m < UPT; ++m) {
-              if (mine(m) && soff[m] < static_cast<uint32_t>(KV_ROPE)) {   // a value unit
-                uint4* q = reinterpret_cast<uint4*>(base + soff[m]);
-                *q = cvt_unit(*q);
-              }
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar->v_full[st]);
-        }
+        if (lane == 0) mbar_arrive(&bar->kv_full[(r0 + tile) % kStages]);
       };
       if constexpr (FP16_SRC) {
         // Up to three tiles in flight (copies committed, not yet landed).  A
@@ -419,6 +500,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         // comes after Q.C^T of the newer tiles, so waiting for a slot while
         // holding an unlanded tile would hold up the scores of that tile
         // (3.62 -> 3.43 ms at 4096 queries of 32K context).
+        auto slot_free = [&](int tile) {
+          const int r = r0 + tile;
+          const bool f = mbar_test(smem_u32(&bar->kv_empty[r % kStages]), ((r / kStages) & 1) ^ 1);
+          return __shfl_sync(0xffffffffu, f, 0);   // lane 0 decides for the warp
+        };
         constexpr int kAhead = 3;
         int n_issued = 0;
         for (int n_landed = 0; ok && n_landed < n_tiles;) {
@@ -443,7 +529,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         // ahead in program order -- land tile i, convert tile i-1, then wait
         // for tile i+2's slot.  (The fp16 schedule above measured slower here:
         // 82 -> 86 us for 64 decode tokens, tile 2's gather waiting for the
-        // conversion of tile 0.)
+        // conversion of tile 0.)  Q.C^T reads the tile as bf16 (exact
+        // products, like fp16); once it has, the value part (units 0..31)
+        // becomes fp16 in place for P.V.
+        auto convert = [&](int tile) {
+          const int r = r0 + tile, st = r % kStages;
+          if (ok && !mbar_wait(&bar->qk_done[st], (r / kStages) & 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 313, r);
+            ok = false;
+          }
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok) {
+            uint8_t* base = sKV + st * KV_STAGE;
+#pragma unroll
+            for (int m = 0; m < UPT; ++m) {
+              if (mine(m) && soff[m] < static_cast<uint32_t>(KV_ROPE)) {   // a value unit
+                uint4* q = reinterpret_cast<uint4*>(base + soff[m]);
+                *q = cvt_unit(*q);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->v_full[st]);
+        };
         issue(0);
         if (n_tiles > 1) issue(1);
         for (int i = 0; ok && i < n_tiles; ++i) {
@@ -458,69 +567,109 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
         if (ok) convert(n_tiles - 1);
       }
-      cp_async_wait<0>();
+      ring += n_tiles;
     }
+    cp_async_wait<0>();
     cluster_wait();
   } else if (warp == C::MMA_WARP) {
     setmaxnreg_dec<C::REG_LOW>();
     // ----------------------------------------------------------- MMA issuer --
-    if (n_tiles > 0 && elect_one()) {
+    if (elect_one()) {
       // Q.C^T in the source's type (bf16 Q in TMEM for a bf16 cache), P.V in fp16
       constexpr uint32_t kQkFmt = FP16_SRC ? 0u : kFmtBF16;
       constexpr uint32_t idesc_qk = idesc_f32acc(kQkFmt, kQkFmt, 128, 64, 0, 0);   // K-major
       constexpr uint32_t idesc_pv = idesc_f32acc(0, 0, 128, 256, 0, 1);    // P K-major, V MN-major
-      bool ok = mbar_wait(&bar->q_full, 0, p.budget);
-      if (!ok) report_error(p.err, kDevErrTimeout, 320, 0);
-      // QK^T runs two tiles ahead of PV: the softmax reads S(i+1) while it
-      // still works on tile i, so S(i+2) can be computed meanwhile.
-      for (int i = 0; ok && i < n_tiles + 2; ++i) {
-        if (i < n_tiles) {
-          const int st = i % kStages;
-          if (!mbar_wait(&bar->kv_full[st], (i / kStages) & 1, p.budget) ||
-              (i > 0 && !mbar_wait(&bar->s_empty, (i - 1) & 1, p.budget))) {
-            report_error(p.err, kDevErrTimeout, 321, i);
+      int ring = 0, G = 0, qc = 0;   // ring jobs, tiles, Q slices so far
+      for (int k = 0;; ++k) {
+        const int w = pair + k * n_pairs;
+        if (w >= n_items) break;
+        if (!mbar_wait(&bar->meta_full[k & 1], (k >> 1) & 1, p.budget)) {
+          report_error(p.err, kDevErrTimeout, 324, k);
+          break;
+        }
+        const int n_tiles = (meta[k & 1].last + 1 + kTileKeys - 1) / kTileKeys;
+        if (meta[k & 1].has_q) {
+          if (!mbar_wait(&bar->q_full, qc & 1, p.budget)) {
+            report_error(p.err, kDevErrTimeout, 320, k);
             break;
           }
-          tc_fence_after();
-          const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
+          // the Q slice is in TMEM: the softmax warps may convert the next
+          // one once this phase has been seen, and its two ring stages are free
+          // (bf16: their Q.C^T phase is closed too, keeping the per-stage
+          // phases in step)
+          mbar_arrive(&bar->q_free);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              umma_f16_ts(tmem + TM_S, tmem + TM_Q + c * 32 + k * 8,
-                          smem_desc(kv_addr + c * 8192 + k * 32, 16, 1024, kSwizzle128B), idesc_qk,
-                          (c | k) ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            const int st = (ring + h) % kStages;
+            if constexpr (!FP16_SRC) mbar_arrive(&bar->qk_done[st]);
+            mbar_arrive(&bar->kv_empty[st]);
+          }
+          ring += 2;
+          ++qc;
+        }
+        if (n_tiles == 0) continue;
+        // QK^T runs two tiles ahead of PV: the softmax reads S(i+1) while it
+        // still works on tile i, so S(i+2) can be computed meanwhile.  Across
+        // items the last two P.V of an item come before the next item's first
+        // Q.C^T, which waits for the next Q slice (converted by the softmax
+        // warps only once this item's tile loop is over).
+        bool ok = true;
+        for (int i = 0; ok && i < n_tiles + 2; ++i) {
+          if (i < n_tiles) {
+            const int r = ring + i, st = r % kStages, gt = G + i;
+            if (!mbar_wait(&bar->kv_full[st], (r / kStages) & 1, p.budget) ||
+                (gt > 0 && !mbar_wait(&bar->s_empty, (gt - 1) & 1, p.budget))) {
+              report_error(p.err, kDevErrTimeout, 321, gt);
+              ok = false;
+              break;
             }
-          }
+            tc_fence_after();
+            const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            umma_f16_ts(tmem + TM_S, tmem + TM_Q + 128 + k * 8,
-                        smem_desc(kv_addr + KV_ROPE + k * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
-          }
-          umma_commit(&bar->s_full);
-          if constexpr (!FP16_SRC) umma_commit(&bar->qk_done[st]);
-        }
-        if (i >= 2) {
-          const int j = i - 2;
-          if (!mbar_wait(&bar->p_full, j & 1, p.budget)) {
-            report_error(p.err, kDevErrTimeout, 322, j);
-            break;
-          }
-          const int st = j % kStages;
-          if (!FP16_SRC && !mbar_wait(&bar->v_full[st], (j / kStages) & 1, p.budget)) {
-            report_error(p.err, kDevErrTimeout, 323, j);
-            break;
-          }
-          tc_fence_after();
-          const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
+            for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            umma_f16_ts(tmem + TM_O, tmem + TM_P + k * 8,
-                        smem_desc(kv_addr + k * 2048, 8192, 1024, kSwizzle128B), idesc_pv, (j | k) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                umma_f16_ts(tmem + TM_S, tmem + TM_Q + c * 32 + kk * 8,
+                            smem_desc(kv_addr + c * 8192 + kk * 32, 16, 1024, kSwizzle128B), idesc_qk,
+                            (c | kk) ? 1u : 0u);
+              }
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              umma_f16_ts(tmem + TM_S, tmem + TM_Q + 128 + kk * 8,
+                          smem_desc(kv_addr + KV_ROPE + kk * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
+            }
+            umma_commit(&bar->s_full);
+            if constexpr (!FP16_SRC) umma_commit(&bar->qk_done[st]);
           }
-          umma_commit(&bar->pv_done);
-          umma_commit(&bar->kv_empty[st]);
+          if (i >= 2) {
+            const int j = i - 2;
+            const int r = ring + j, st = r % kStages, gt = G + j;
+            if (!mbar_wait(&bar->p_full, gt & 1, p.budget)) {
+              report_error(p.err, kDevErrTimeout, 322, gt);
+              ok = false;
+              break;
+            }
+            if (!FP16_SRC && !mbar_wait(&bar->v_full[st], (r / kStages) & 1, p.budget)) {
+              report_error(p.err, kDevErrTimeout, 323, gt);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kv_addr = smem_u32(sKV + st * KV_STAGE);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_f16_ts(tmem + TM_O, tmem + TM_P + kk * 8,
+                          smem_desc(kv_addr + kk * 2048, 8192, 1024, kSwizzle128B), idesc_pv,
+                          (j | kk) ? 1u : 0u);
+            }
+            umma_commit(&bar->pv_done);
+            umma_commit(&bar->kv_empty[st]);
+          }
         }
+        if (!ok) break;
+        ring += n_tiles;
+        G += n_tiles;
       }
     }
     cluster_wait();
@@ -546,8 +695,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     const uint32_t x_free_remote = mapa_shared(smem_u32(&bar->x_free[sw]), peer);
     const float NEG_INF = __int_as_float(0xff800000);
     const float scale = p.scale_log2;
-    float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
-    float l_runA = 0.f, l_runB = 0.f;           // this lane's share of the row sums
     bool ok = true;
     // bounded wait polled by every lane (each lane acquires for itself); the
     // vote makes the outcome warp-uniform.  On an already completed phase this
@@ -558,9 +705,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       if (!all && lane == 0) report_error(p.err, kDevErrTimeout, site, info);
       return all;
     };
-    // S(t) of this warp's 16 heads, this CTA's fp32 partial over its 288 dims:
-    // s[4k], s[4k+1] = head rA, keys 8k+ku, 8k+ku+1; s[4k+2], s[4k+3] = head rB.
-    // Split in two so the TMEM load's latency overlaps other work.
+    // S of global tile t, this warp's 16 heads, this CTA's fp32 partial over
+    // its 288 dims: s[4k], s[4k+1] = head rA, keys 8k+ku, 8k+ku+1; s[4k+2],
+    // s[4k+3] = head rB.  Split in two so the TMEM load's latency overlaps
+    // other work.
     auto load_s_issue = [&](int t, uint32_t (&s)[32]) -> bool {
       if (!wwait(&bar->s_full, t & 1, false, 330, t)) return false;
       tc_fence_after();
@@ -590,23 +738,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       if (lane == 0) bulk_copy_to_peer(x_base_remote, stg_base, XBLK, x_full_remote);
       return true;
     };
-
-    // every softmax warp waits for the Q slice, also when there is nothing to
-    // attend, so no TMA write is still in flight when the CTA exits
-    if (!wwait(&bar->q_tma, 0, false, 338, 0)) ok = false;
-    if (n_tiles > 0) {
-      // Q_r row h into TMEM (shape .32x32b: lane = head): warps of the first
-      // warpgroup write dims [0, 144) of the CTA's 288, the second [144, 288)
+    // The Q slice of the item whose Q jobs are ring jobs rq, rq + 1 -> TMEM
+    // (shape .32x32b: lane = head): warps of the first warpgroup write dims
+    // [0, 144) of the CTA's 288, the second [144, 288).  Stage A holds latent
+    // boxes 0-1 and RoPE rows 0-63, stage B boxes 2-3 and RoPE rows 64-127.
+    int qn = 0;   // Q slices converted so far
+    auto convert_q = [&](int rq, int info) -> bool {
+      const int sa = rq % kStages, sb = (rq + 1) % kStages;
+      // the MMA thread has seen the previous slice's q_full phase (so this
+      // slice's arrivals cannot run a phase ahead of it), and the slice landed
+      if ((qn > 0 && !wwait(&bar->q_free, (qn - 1) & 1, false, 337, info)) ||
+          !wwait(&bar->kv_full[sa], (rq / kStages) & 1, false, 338, info) ||
+          !wwait(&bar->kv_full[sb], ((rq + 1) / kStages) & 1, false, 338, info))
+        return false;
+      const uint8_t* qa = sKV + sa * KV_STAGE;
+      const uint8_t* qb = sKV + sb * KV_STAGE;
       const int g = sw >> 2;
       const int h = static_cast<int>(quarter * 32 + lane);
+      const int hl = h & 63;
       uint32_t qv[72];
 #pragma unroll
       for (int m = 0; m < 18; ++m) {
         const int u = 18 * g + m;        // unit of the CTA's 288 dims: 0..31 latent, 32..35 RoPE
-        const uint32_t off = u < 32 ? (u >> 3) * kQBox + h * 128 + (((u & 7) ^ (h & 7)) << 4)
-                                    : 4 * kQBox + h * 64 + (((u - 32) ^ ((h >> 1) & 3)) << 4);
+        const uint8_t* src;
+        if (u < 32) {
+          const int c = u >> 3;
+          src = ((c >> 1) ? qb : qa) + (c & 1) * kQBox + h * 128 + (((u & 7) ^ (h & 7)) << 4);
+        } else {
+          src = ((h >> 6) ? qb : qa) + 2 * kQBox + hl * 64 + (((u - 32) ^ ((hl >> 1) & 3)) << 4);
+        }
         uint4 raw = make_uint4(0, 0, 0, 0);
-        if (ok && h < H) raw = *reinterpret_cast<const uint4*>(sQ + off);
+        if (h < H) raw = *reinterpret_cast<const uint4*>(src);
         const uint4 v = FP16_SRC ? cvt_unit(raw) : raw;   // Q in the type of the gathered entries
         qv[4 * m + 0] = v.x;
         qv[4 * m + 1] = v.y;
@@ -631,236 +793,328 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->q_full);
-    }
+      ++qn;
+      return true;
+    };
+
     cluster_wait();          // the peer's barriers exist: exchanges may start
 
-    uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
-    if (n_tiles > 0) {
-      ok = ok && load_s_issue(0, cur);
-      if (ok) {
-        load_s_finish();
-        ok = send(0, cur);
-      }
-    }
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      // 1. start loading the next tile's partial scores; they are shipped to
-      //    the peer once this tile's scores are assembled
-      const bool more = i + 1 < n_tiles;
-      uint32_t snext[32];
-      if (more && !load_s_issue(i + 1, snext)) {
+    int G = 0, ring = 0, ke = 0;   // tiles, ring jobs, epilogues so far
+    bool have_q = false;           // this item's Q slice is already in TMEM
+    for (int k = 0; ok; ++k) {
+      const int w = pair + k * n_pairs;
+      if (w >= n_items) break;
+      if (!wwait(&bar->meta_full[k & 1], (k >> 1) & 1, false, 336, k)) {
         ok = false;
         break;
       }
-      // 2. the peer's partial scores of tile i (this warp's own barrier)
-      if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[sw], XBLK);
-      if (!wwait(&bar->x_full[sw], i & 1, true, 332, i)) {
-        ok = false;
-        break;
+      // the item's metadata in registers: the buffer is restaged for item k + 2
+      // once this warp's tile loop is over
+      const ItemMeta it = meta[k & 1];
+      const int n_tiles = (it.last + 1 + kTileKeys - 1) / kTileKeys;
+      const uint32_t* sV = sValid + (k & 1) * 64;
+      if (it.has_q) {
+        if (!have_q && !convert_q(ring, k)) {
+          ok = false;
+          break;
+        }
+        ring += 2;
       }
-      uint32_t xp[32];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(xp[4 * q]), "=r"(xp[4 * q + 1]), "=r"(xp[4 * q + 2]), "=r"(xp[4 * q + 3])
-                     : "r"(x_base + q * 512 + lane * 16)
-                     : "memory");
+      float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
+      float l_runA = 0.f, l_runB = 0.f;           // this lane's share of the row sums
+      uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
+      if (n_tiles > 0) {
+        ok = load_s_issue(G, cur);
+        if (ok) {
+          load_s_finish();
+          ok = send(G, cur);
+        }
       }
-      // own + peer partial in fp32 (f32x2 pairs; each lane the IEEE fp32 add):
-      // the peer computes peer + own, the same sum
-      float sv[32];
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int gt = G + i;
+        // 1. start loading the next tile's partial scores; they are shipped to
+        //    the peer once this tile's scores are assembled
+        const bool more = i + 1 < n_tiles;
+        uint32_t snext[32];
+        if (more && !load_s_issue(gt + 1, snext)) {
+          ok = false;
+          break;
+        }
+        // 2. the peer's partial scores of tile i (this warp's own barrier)
+        if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[sw], XBLK);
+        if (!wwait(&bar->x_full[sw], gt & 1, true, 332, gt)) {
+          ok = false;
+          break;
+        }
+        uint32_t xp[32];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float2 v = unpack_f32x2(add_f32x2(pack_f32x2(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
-                                                pack_f32x2(__uint_as_float(xp[2 * c]), __uint_as_float(xp[2 * c + 1]))));
-        sv[2 * c] = v.x;
-        sv[2 * c + 1] = v.y;
-      }
-      __syncwarp();
-      // the values are in registers: the peer may refill the buffer
-      if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote);
-      // 3. mask positions past the selection / padding: key 8k + ku + e
-      const uint64_t vmask = static_cast<uint64_t>(sValid[2 * i]) | (static_cast<uint64_t>(sValid[2 * i + 1]) << 32);
-      if (vmask != ~uint64_t(0)) {
+        for (int q = 0; q < 8; ++q) {
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(xp[4 * q]), "=r"(xp[4 * q + 1]), "=r"(xp[4 * q + 2]), "=r"(xp[4 * q + 3])
+                       : "r"(x_base + q * 512 + lane * 16)
+                       : "memory");
+        }
+        // own + peer partial in fp32 (f32x2 pairs; each lane the IEEE fp32 add):
+        // the peer computes peer + own, the same sum
+        float sv[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int c = 0; c < 16; ++c) {
+          const float2 v = unpack_f32x2(add_f32x2(pack_f32x2(__uint_as_float(cur[2 * c]), __uint_as_float(cur[2 * c + 1])),
+                                                  pack_f32x2(__uint_as_float(xp[2 * c]), __uint_as_float(xp[2 * c + 1]))));
+          sv[2 * c] = v.x;
+          sv[2 * c + 1] = v.y;
+        }
+        __syncwarp();
+        // the values are in registers: the peer may refill the buffer
+        if (lane == 0) mbar_arrive_remote_relaxed(x_free_remote);
+        // 3. mask positions past the selection / padding: key 8k + ku + e
+        const uint64_t vmask = static_cast<uint64_t>(sV[2 * i]) | (static_cast<uint64_t>(sV[2 * i + 1]) << 32);
+        if (vmask != ~uint64_t(0)) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            if (!((vmask >> (8 * k + ku + e)) & 1u)) {
-              sv[4 * k + e] = NEG_INF;
-              sv[4 * k + 2 + e] = NEG_INF;
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              if (!((vmask >> (8 * kk + ku + e)) & 1u)) {
+                sv[4 * kk + e] = NEG_INF;
+                sv[4 * kk + 2 + e] = NEG_INF;
+              }
             }
           }
         }
-      }
-      // 4. row maxima over the 64 columns: 16 per lane, then the lane group
-      float mA = fmaxf(sv[0], sv[1]), mB = fmaxf(sv[2], sv[3]);
+        // 4. row maxima over the 64 columns: 16 per lane, then the lane group
+        float mA = fmaxf(sv[0], sv[1]), mB = fmaxf(sv[2], sv[3]);
 #pragma unroll
-      for (int k = 1; k < 8; ++k) {
-        mA = fmaxf(mA, fmaxf(sv[4 * k], sv[4 * k + 1]));
-        mB = fmaxf(mB, fmaxf(sv[4 * k + 2], sv[4 * k + 3]));
-      }
+        for (int kk = 1; kk < 8; ++kk) {
+          mA = fmaxf(mA, fmaxf(sv[4 * kk], sv[4 * kk + 1]));
+          mB = fmaxf(mB, fmaxf(sv[4 * kk + 2], sv[4 * kk + 3]));
+        }
 #pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, o));
-        mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, o));
-      }
-      float alphaA = 1.f, alphaB = 1.f;
-      bool grow = false;
-      {
-        const float nA = fmaxf(m_runA, mA * scale), nB = fmaxf(m_runB, mB * scale);
-        if (nA > m_runA + 8.0f) {                      // true on the first finite tile
-          alphaA = fast_exp2(m_runA - nA);             // exp2(-inf) = 0
-          m_runA = nA;
-          grow = true;
+        for (int o = 1; o <= 2; o <<= 1) {
+          mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, o));
+          mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, o));
         }
-        if (nB > m_runB + 8.0f) {
-          alphaB = fast_exp2(m_runB - nB);
-          m_runB = nB;
-          grow = true;
+        float alphaA = 1.f, alphaB = 1.f;
+        bool grow = false;
+        {
+          const float nA = fmaxf(m_runA, mA * scale), nB = fmaxf(m_runB, mB * scale);
+          if (nA > m_runA + 8.0f) {                      // true on the first finite tile
+            alphaA = fast_exp2(m_runA - nA);             // exp2(-inf) = 0
+            m_runA = nA;
+            grow = true;
+          }
+          if (nB > m_runB + 8.0f) {
+            alphaB = fast_exp2(m_runB - nB);
+            m_runB = nB;
+            grow = true;
+          }
         }
+        const float refA = m_runA == NEG_INF ? 0.f : m_runA;
+        const float refB = m_runB == NEG_INF ? 0.f : m_runB;
+        // next tile's partial scores: wait for the TMEM load, ship
+        if (more) {
+          load_s_finish();
+          if (!send(gt + 1, snext)) {
+            ok = false;
+            break;
+          }
+        }
+        // 5. probabilities (fp16 pairs, in the .16x128b order of P's columns) and row sums
+        // (exponent arguments and row sums on f32x2 pairs: half the FMA/add
+        // instructions; each lane is the fp32 operation of the scalar form)
+        uint32_t pk[16];
+        const uint64_t sc2 = pack_f32x2(scale, scale);
+        const uint64_t nA2 = pack_f32x2(-refA, -refA), nB2 = pack_f32x2(-refB, -refB);
+        uint64_t sA2 = 0ull, sB2 = 0ull;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const float2 xa = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * kk], sv[4 * kk + 1]), sc2, nA2));
+          const float2 xb = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * kk + 2], sv[4 * kk + 3]), sc2, nB2));
+          const float a0 = fast_exp2(xa.x), a1 = fast_exp2(xa.y);
+          const float b0 = fast_exp2(xb.x), b1 = fast_exp2(xb.y);
+          sA2 = add_f32x2(sA2, pack_f32x2(a0, a1));
+          sB2 = add_f32x2(sB2, pack_f32x2(b0, b1));
+          pk[2 * kk] = pack_half2(a0, a1);
+          pk[2 * kk + 1] = pack_half2(b0, b1);
+        }
+        const float2 sa = unpack_f32x2(sA2), sb = unpack_f32x2(sB2);
+        l_runA = l_runA * alphaA + (sa.x + sa.y);
+        l_runB = l_runB * alphaB + (sb.x + sb.y);
+        // 6. PV(i-1) must be done before P and O are touched (the previous
+        //    item's last P.V was waited for by its epilogue)
+        if (i > 0 && !wwait(&bar->pv_done, (gt - 1) & 1, false, 333, gt)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              o[4 * kk] = __float_as_uint(__uint_as_float(o[4 * kk]) * alphaA);
+              o[4 * kk + 1] = __float_as_uint(__uint_as_float(o[4 * kk + 1]) * alphaA);
+              o[4 * kk + 2] = __float_as_uint(__uint_as_float(o[4 * kk + 2]) * alphaB);
+              o[4 * kk + 3] = __float_as_uint(__uint_as_float(o[4 * kk + 3]) * alphaB);
+            }
+            tmem_st_16x256b_x8(tbase + TM_O + 64 * c, o);
+          }
+        }
+        tmem_st_16x128b_x8(tbase + TM_P, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->p_full);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) cur[c] = snext[c];
       }
-      const float refA = m_runA == NEG_INF ? 0.f : m_runA;
-      const float refB = m_runB == NEG_INF ? 0.f : m_runB;
-      // next tile's partial scores: wait for the TMEM load, ship
-      if (more) {
-        load_s_finish();
-        if (!send(i + 1, snext)) {
+      if (!ok) break;
+      // the validity bits of this parity may be restaged (item k + 2)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->meta_free[k & 1]);
+      ring += n_tiles;
+      // The next item's Q slice into TMEM now -- every Q.C^T issued so far has
+      // completed (this warp loaded its scores) -- so that item's first Q.C^T
+      // runs during this epilogue.
+      have_q = false;
+      if (w + n_pairs < n_items) {
+        if (!wwait(&bar->meta_full[(k + 1) & 1], ((k + 1) >> 1) & 1, false, 336, k + 1)) {
           ok = false;
           break;
         }
       }
-      // 5. probabilities (fp16 pairs, in the .16x128b order of P's columns) and row sums
-      // (exponent arguments and row sums on f32x2 pairs: half the FMA/add
-      // instructions; each lane is the fp32 operation of the scalar form)
-      uint32_t pk[16];
-      const uint64_t sc2 = pack_f32x2(scale, scale);
-      const uint64_t nA2 = pack_f32x2(-refA, -refA), nB2 = pack_f32x2(-refB, -refB);
-      uint64_t sA2 = 0ull, sB2 = 0ull;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float2 xa = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * k], sv[4 * k + 1]), sc2, nA2));
-        const float2 xb = unpack_f32x2(fma_f32x2(pack_f32x2(sv[4 * k + 2], sv[4 * k + 3]), sc2, nB2));
-        const float a0 = fast_exp2(xa.x), a1 = fast_exp2(xa.y);
-        const float b0 = fast_exp2(xb.x), b1 = fast_exp2(xb.y);
-        sA2 = add_f32x2(sA2, pack_f32x2(a0, a1));
-        sB2 = add_f32x2(sB2, pack_f32x2(b0, b1));
-        pk[2 * k] = pack_half2(a0, a1);
-        pk[2 * k + 1] = pack_half2(b0, b1);
-      }
-      const float2 sa = unpack_f32x2(sA2), sb = unpack_f32x2(sB2);
-      l_runA = l_runA * alphaA + (sa.x + sa.y);
-      l_runB = l_runB * alphaB + (sb.x + sb.y);
-      // 6. PV(i-1) must be done before P and O are touched
-      if (i > 0 && !wwait(&bar->pv_done, (i - 1) & 1, false, 333, i)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (i > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alphaA);
-            o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alphaA);
-            o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alphaB);
-            o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alphaB);
-          }
-          tmem_st_16x256b_x8(tbase + TM_O + 64 * c, o);
+      if (w + n_pairs < n_items && meta[(k + 1) & 1].has_q) {
+        if (!convert_q(ring, k + 1)) {
+          ok = false;
+          break;
         }
+        have_q = true;
       }
-      tmem_st_16x128b_x8(tbase + TM_P, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->p_full);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) cur[c] = snext[c];
-    }
 
-    // ---- epilogue: O / l -> bf16 (or fp32 partial) ----
-    if (ok && n_tiles > 0 && !wwait(&bar->pv_done, (n_tiles - 1) & 1, false, 335, n_tiles)) ok = false;
-    tc_fence_after();
+      // ---- epilogue: O / l -> bf16 (or fp32 partial); nothing for a row that
+      // lies in no sequence ----
+      if (it.status != 302) {
+        if (n_tiles > 0 && !wwait(&bar->pv_done, (G + n_tiles - 1) & 1, false, 335, G + n_tiles)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float lA = l_runA, lB = l_runB;
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      l_runA += __shfl_xor_sync(0xffffffffu, l_runA, o);
-      l_runB += __shfl_xor_sync(0xffffffffu, l_runB, o);
-    }
-    const bool anyA = n_tiles > 0 && l_runA > 0.f, anyB = n_tiles > 0 && l_runB > 0.f;
-    const float invA = anyA ? 1.f / l_runA : 0.f, invB = anyB ? 1.f / l_runB : 0.f;
-    const float lseA = anyA ? (m_runA + __log2f(l_runA)) * 0.69314718055994531f : NEG_INF;
-    const float lseB = anyB ? (m_runB + __log2f(l_runB)) * 0.69314718055994531f : NEG_INF;
-    // O chunk c (64 of the CTA's 256 value dims) of this warp's 16 heads
-    auto load_o = [&](int c, uint32_t (&o)[32]) {
-      if (n_tiles > 0) {
-        tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = 0u;
-      }
-    };
-    if (p.nsplit == 1) {
-      // O / l as bf16 into ring stages 0-1 (idle now) in the 128-byte-swizzled
-      // layout of four [H x 64-dim] TMA boxes, then one thread stores the boxes:
-      // whole rows leave the SM instead of pieces strided by a head row.
-      uint8_t* sO = sKV;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        load_o(c, o);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          // dims 64c + 8k + ku, +1: box c, 16-byte unit k, byte 2*ku
-          if (hA < H) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[4 * k]) * invA,
-                                                           __uint_as_float(o[4 * k + 1]) * invA);
-            *reinterpret_cast<__nv_bfloat162*>(sO + c * kQBox + hA * 128 + ((k ^ (hA & 7)) << 4) + 2 * ku) = v;
+        for (int o = 1; o <= 2; o <<= 1) {
+          lA += __shfl_xor_sync(0xffffffffu, lA, o);
+          lB += __shfl_xor_sync(0xffffffffu, lB, o);
+        }
+        const bool anyA = n_tiles > 0 && lA > 0.f, anyB = n_tiles > 0 && lB > 0.f;
+        const float invA = anyA ? 1.f / lA : 0.f, invB = anyB ? 1.f / lB : 0.f;
+        const float lseA = anyA ? (m_runA + __log2f(lA)) * 0.69314718055994531f : NEG_INF;
+        const float lseB = anyB ? (m_runB + __log2f(lB)) * 0.69314718055994531f : NEG_INF;
+        if (p.nsplit == 1) {
+          // Each lane stores whole 64-byte runs of one head: the inverse row
+          // sums go through shared memory to the .32x32b layout (lane = head),
+          // the two warps of a lane quarter taking 128 value dims each.
+          float* inv_s = sInv + (ke & 1) * 128;
+          if ((lane & 3u) == 0) {
+            inv_s[hA] = invA;
+            inv_s[hB] = invB;
           }
-          if (hB < H) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[4 * k + 2]) * invB,
-                                                           __uint_as_float(o[4 * k + 3]) * invB);
-            *reinterpret_cast<__nv_bfloat162*>(sO + c * kQBox + hB * 128 + ((k ^ (hB & 7)) << 4) + 2 * ku) = v;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->red);
+          if (!wwait(&bar->red, ke & 1, false, 339, ke)) {
+            ok = false;
+            break;
+          }
+          // This warp's 4 KB staging block transposes the stores: our last
+          // bulk copy out of it has been read once the peer arrived on x_free
+          // for the last tile we sent.
+          const int t_last = G + n_tiles - 1;
+          if (t_last >= 0 && !wwait(&bar->x_free[sw], t_last & 1, true, 334, t_last)) {
+            ok = false;
+            break;
+          }
+          const int h = static_cast<int>(quarter * 32 + lane);
+          const float inv = inv_s[h];
+          const int cb = 128 * (sw >> 2);   // this warp's 128 of the CTA's 256 value dims
+          // row r of the block: head 32q + r, 64 dims = 8 units, unit u at (u ^ (r & 7)) * 16
+          const uint32_t blk = stg_base;
+          uint16_t* obase = p.out + (static_cast<int64_t>(it.row) * H + quarter * 32) * 512 + rank * 256 + cb;
+#pragma unroll 1
+          for (int j = 0; j < 2; ++j) {
+            uint32_t o0[32], o1[32];
+            if (n_tiles > 0) {
+              tmem_ld32(tmem + ((quarter * 32u) << 16) + TM_O + cb + 64 * j, o0);
+              tmem_ld32(tmem + ((quarter * 32u) << 16) + TM_O + cb + 64 * j + 32, o1);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o0[e] = o1[e] = 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = 8 * (u & 3) + 2 * e;   // column pair inside o0 (u < 4) or o1
+                const float x0 = __uint_as_float(u < 4 ? o0[c] : o1[c]) * inv;
+                const float x1 = __uint_as_float(u < 4 ? o0[c + 1] : o1[c + 1]) * inv;
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                wv[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(blk + lane * 128 + ((u ^ (lane & 7)) << 4)),
+                           "r"(wv[0]), "r"(wv[1]), "r"(wv[2]), "r"(wv[3])
+                           : "memory");
+            }
+            __syncwarp();
+            // eight lanes per head row: each store instruction writes four whole 128-byte runs
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + static_cast<int>(lane >> 3), uu = static_cast<int>(lane & 7u);
+              uint4 val;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                           : "r"(blk + r * 128 + ((uu ^ (r & 7)) << 4))
+                           : "memory");
+              if (static_cast<int>(quarter) * 32 + r < H)
+                *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(r) * 512 + 64 * j + 8 * uu) = val;
+            }
+            __syncwarp();
+          }
+          if (rank == 0 && (lane & 3u) == 0 && p.lse != nullptr) {
+            if (hA < H) p.lse[static_cast<int64_t>(it.row) * H + hA] = lseA;
+            if (hB < H) p.lse[static_cast<int64_t>(it.row) * H + hB] = lseB;
+          }
+          ++ke;
+        } else {
+          const int64_t prow = (static_cast<int64_t>(it.row) * p.nsplit + it.split) * 128;
+          float* oA = p.part_o + (prow + hA) * 512 + rank * 256 + ku;
+          float* oB = p.part_o + (prow + hB) * 512 + rank * 256 + ku;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            if (n_tiles > 0) {
+              tmem_ld_16x256b_x8(tbase + TM_O + 64 * c, o);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = 0u;
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              *reinterpret_cast<float2*>(oA + 64 * c + 8 * kk) =
+                  make_float2(__uint_as_float(o[4 * kk]) * invA, __uint_as_float(o[4 * kk + 1]) * invA);
+              *reinterpret_cast<float2*>(oB + 64 * c + 8 * kk) =
+                  make_float2(__uint_as_float(o[4 * kk + 2]) * invB, __uint_as_float(o[4 * kk + 3]) * invB);
+            }
+          }
+          if ((lane & 3u) == 0) {        // each value half with its own log-sum-exp
+            p.part_lse[(prow * 2 + rank * 128) + hA] = lseA;
+            p.part_lse[(prow * 2 + rank * 128) + hB] = lseB;
           }
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&bar->red);
-      const bool staged = wwait(&bar->red, 0, false, 339, n_tiles);
-      if (staged && sw == 0 && lane == 0) {
-#pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          tma_store_2d(&maps.out, sO + bx * kQBox, static_cast<int>(rank) * 256 + bx * 64, row * H);
-        bulk_commit_group();
-        bulk_wait_read_all();    // the CTA may leave once the boxes are read
-      }
-      if (rank == 0 && (lane & 3u) == 0 && p.lse != nullptr) {
-        if (hA < H) p.lse[static_cast<int64_t>(row) * H + hA] = lseA;
-        if (hB < H) p.lse[static_cast<int64_t>(row) * H + hB] = lseB;
-      }
-    } else {
-      const int64_t prow = (static_cast<int64_t>(row) * p.nsplit + split) * 128;
-      float* oA = p.part_o + (prow + hA) * 512 + rank * 256 + ku;
-      float* oB = p.part_o + (prow + hB) * 512 + rank * 256 + ku;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        load_o(c, o);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          *reinterpret_cast<float2*>(oA + 64 * c + 8 * k) =
-              make_float2(__uint_as_float(o[4 * k]) * invA, __uint_as_float(o[4 * k + 1]) * invA);
-          *reinterpret_cast<float2*>(oB + 64 * c + 8 * k) =
-              make_float2(__uint_as_float(o[4 * k + 2]) * invB, __uint_as_float(o[4 * k + 3]) * invB);
-        }
-      }
-      if ((lane & 3u) == 0) {        // each value half with its own log-sum-exp
-        p.part_lse[(prow * 2 + rank * 128) + hA] = lseA;
-        p.part_lse[(prow * 2 + rank * 128) + hB] = lseB;
-      }
+      G += n_tiles;
     }
   }
   tc_fence_before();
@@ -919,12 +1173,41 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   }
 }
 
+// CTA pairs of the kernel that can be resident at once on this device (an
+// occupancy query, cached per device and variant): a persistent pair that
+// waited for a free slot would start after the others had finished.
 template <bool FP16_SRC>
-cudaError_t launch_variant(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+int resident_pairs() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v != 0) return v - 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(kSmem);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_kernel<FP16_SRC>, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();   // a refused query leaves no sticky error behind
+  cache[dev].store(n + 1, std::memory_order_relaxed);
+  return n;
+}
+
+template <bool FP16_SRC>
+cudaError_t launch_variant(const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+  const int64_t items = static_cast<int64_t>(p.total_q) * p.nsplit;
+  if (items <= 0) return cudaSuccess;
   cudaError_t e =
       cudaFuncSetAttribute(sparse_mla_kernel<FP16_SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  sparse_mla_kernel<FP16_SRC><<<grid, Cfg::THREADS, kSmem, stream>>>(p, maps);
+  int pairs = resident_pairs<FP16_SRC>();
+  if (pairs < 1) pairs = sm_count() / 2;
+  if (pairs < 1) pairs = 1;
+  const int cap = mla_pair_cap();
+  if (cap > 0 && cap < pairs) pairs = cap;
+  if (items < pairs) pairs = static_cast<int>(items);
+  sparse_mla_kernel<FP16_SRC><<<dim3(static_cast<unsigned>(2 * pairs)), Cfg::THREADS, kSmem, stream>>>(p, maps);
   return cudaGetLastError();
 }
 
@@ -961,12 +1244,12 @@ bool mla_use_fp16_copy(int total_q, int max_kv_len, int64_t total_keys, int k_se
 
 size_t mla_smem_bytes() { return kSmem; }
 
-cudaError_t launch_sparse_mla(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
-  return launch_variant<false>(grid, p, maps, stream);
+cudaError_t launch_sparse_mla(const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+  return launch_variant<false>(p, maps, stream);
 }
 
-cudaError_t launch_sparse_mla_fp16(dim3 grid, const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
-  return launch_variant<true>(grid, p, maps, stream);
+cudaError_t launch_sparse_mla_fp16(const MlaParams& p, const MlaMaps& maps, cudaStream_t stream) {
+  return launch_variant<true>(p, maps, stream);
 }
 
 cudaError_t launch_latent_to_fp16(const uint16_t* src, uint16_t* dst, int64_t n_elems, cudaStream_t stream) {
