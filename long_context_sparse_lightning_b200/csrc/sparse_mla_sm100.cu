@@ -199,7 +199,7 @@ __device__ __forceinline__ uint32_t tile_unit_offset(int j, int u) {
 // recomputing it with dependent global loads.
 struct ItemMeta {
   int32_t last;     // last valid slot of the selection, -1: none
-  int32_t row, split, status, has_q;
+  int32_t row, split, status;
 };
 static_assert(16 + 2 * sizeof(ItemMeta) <= 64, "item metadata fits the misc area");
 
@@ -209,17 +209,37 @@ static_assert(16 + 2 * sizeof(ItemMeta) <= 64, "item metadata fits the misc area
 // of cu_q (nothing of it is written).
 struct MlaItem {
   int row, split, b, kv, status;
-  int e_begin, e_count;   // the split's slots of the selection (0 slots: nothing to attend)
+  int e_begin, e_count;   // the split's slots of the selection
   int64_t kstart;
-  // the item carries a Q slice through the ring: every role decides this the
-  // same way, before the positions are staged
-  __device__ __forceinline__ bool has_q() const { return e_count > 0; }
 };
 
-__device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int w) {
+// Slots of the selection that split `split` covers.
+__device__ __forceinline__ int split_slots(const MlaParams& p, int split) {
+  const int e_begin = split * p.keys_per_split;
+  return max(0, min(p.k_sel, e_begin + p.keys_per_split) - e_begin);
+}
+
+// Whether item w carries a Q slice through the ring: a function of the launch
+// alone (no loads), so every role decides it at once and alike; an item whose
+// sequence turns out to be invalid still takes (and drops) its slice.
+__device__ __forceinline__ bool item_has_q(const MlaParams& p, int w) { return split_slots(p, w % p.nsplit) > 0; }
+
+// The load-free part of an item: its row and slots.
+__device__ __forceinline__ MlaItem mla_item_base(const MlaParams& p, int w) {
   MlaItem it;
   it.row = w / p.nsplit;
   it.split = w - it.row * p.nsplit;
+  it.e_begin = it.split * p.keys_per_split;
+  it.e_count = split_slots(p, it.split);
+  it.b = 0;
+  it.kv = 0;
+  it.kstart = 0;
+  it.status = 0;
+  return it;
+}
+
+// The row's sequence and its descriptors (dependent loads).
+__device__ __forceinline__ void mla_item_seq(const MlaParams& p, MlaItem& it) {
   // the row's sequence: the last b with cu_q[b] <= row (empty sequences skipped)
   int lo = 0, hi = p.num_seqs - 1;
   while (lo < hi) {
@@ -231,25 +251,15 @@ __device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int w) {
     }
   }
   it.b = lo;
-  it.kv = 0;
-  it.kstart = 0;
-  it.status = 0;
-  it.e_begin = it.split * p.keys_per_split;
-  it.e_count = 0;
   const int q0 = __ldg(&p.cu_q[lo]);
   const int q_len = __ldg(&p.cu_q[lo + 1]) - q0;
   if (q0 < 0 || it.row < q0 || it.row >= q0 + q_len) {
     it.status = 302;
-    return it;
+    return;
   }
   it.kv = __ldg(&p.kv_len[lo]);
   it.kstart = seq_start(p.pt, p.kv_start, lo);
-  if (q_len > it.kv || !seq_rows_ok(p.pt, it.kstart, it.kv, p.total_keys)) {
-    it.status = 301;
-    return it;
-  }
-  it.e_count = max(0, min(p.k_sel, it.e_begin + p.keys_per_split) - it.e_begin);
-  return it;
+  if (q_len > it.kv || !seq_rows_ok(p.pt, it.kstart, it.kv, p.total_keys)) it.status = 301;
 }
 
 // FP16_SRC: p.kv is an fp16 copy of the latent cache (rows land ready for the
@@ -375,13 +385,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
     };
     int ring = 0;           // ring jobs issued so far (Q halves and tiles)
-    MlaItem nxt;            // the next item, fetched while the current one's Q slice is in flight
-    if (pair < n_items) nxt = mla_item(p, pair);
+    // The next item: its row and slots need no loads; its sequence is looked
+    // up while the current item's Q slice is in flight (the first item's while
+    // its own slice and positions are).
+    MlaItem nxt;
+    if (pair < n_items) nxt = mla_item_base(p, pair);
     for (int k = 0; ok; ++k) {
       const int w = pair + k * n_pairs;
       if (w >= n_items) break;
-      const MlaItem it = nxt;
-      if (it.status != 0 && tid == 0 && rank == 0) report_error(p.err, kDevErrBounds, it.status, it.b);
+      MlaItem it = nxt;
       // this item's positions: loads first (one memory latency)
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.row) * p.k_sel + it.e_begin;
       int v[10];
@@ -394,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       // rows 64h..64h+63), issued before the positions are staged so that it
       // lands while the previous item's last tiles are still being processed.
       // Every warp waits for the slot before its arrival.
-      if (it.has_q()) {
+      if (item_has_q(p, w)) {
         const int rope_rows = H < 64 ? H : 64;
         for (int h = 0; ok && h < 2; ++h, ++ring) {
           slot_wait(ring);
@@ -422,7 +434,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
         if (!ok) break;
       }
-      if (w + n_pairs < n_items) nxt = mla_item(p, w + n_pairs);
+      if (k == 0) mla_item_seq(p, it);
+      if (w + n_pairs < n_items) {
+        nxt = mla_item_base(p, w + n_pairs);
+        mla_item_seq(p, nxt);
+      }
+      if (it.status != 0 && tid == 0 && rank == 0) report_error(p.err, kDevErrBounds, it.status, it.b);
       // The previous item's tiles are issued and landed by every warp (sIdx is
       // free), and the validity buffer of this item's parity is free once the
       // softmax warps are done with item k - 2.
@@ -436,7 +453,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         m.row = it.row;
         m.split = it.split;
         m.status = it.status;
-        m.has_q = it.has_q() ? 1 : 0;
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -450,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       for (int q = 0; q < 10; ++q) {
         const int j = tid + q * C::PTHREADS;
         if (j < 2048) {
-          int e = (v[q] < 0 || v[q] >= it.kv) ? -1 : v[q];
+          int e = (it.status != 0 || v[q] < 0 || v[q] >= it.kv) ? -1 : v[q];
           if (e >= 0) {
             const int64_t r = cache_row(p.pt, it.b, it.kstart, e);
             if (r < 0) report_error(p.err, kDevErrBounds, 303, it.b);   // a page id outside the pool: skipped
@@ -588,7 +604,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
           break;
         }
         const int n_tiles = (meta[k & 1].last + 1 + kTileKeys - 1) / kTileKeys;
-        if (meta[k & 1].has_q) {
+        if (item_has_q(p, w)) {
           if (!mbar_wait(&bar->q_full, qc & 1, p.budget)) {
             report_error(p.err, kDevErrTimeout, 320, k);
             break;
@@ -804,6 +820,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     for (int k = 0; ok; ++k) {
       const int w = pair + k * n_pairs;
       if (w >= n_items) break;
+      // the Q slice first: it needs no metadata (the first item's lands while
+      // the producers are still staging its positions)
+      if (item_has_q(p, w)) {
+        if (!have_q && !convert_q(ring, k)) {
+          ok = false;
+          break;
+        }
+        ring += 2;
+      }
       if (!wwait(&bar->meta_full[k & 1], (k >> 1) & 1, false, 336, k)) {
         ok = false;
         break;
@@ -813,13 +838,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       const ItemMeta it = meta[k & 1];
       const int n_tiles = (it.last + 1 + kTileKeys - 1) / kTileKeys;
       const uint32_t* sV = sValid + (k & 1) * 64;
-      if (it.has_q) {
-        if (!have_q && !convert_q(ring, k)) {
-          ok = false;
-          break;
-        }
-        ring += 2;
-      }
       float m_runA = NEG_INF, m_runB = NEG_INF;   // running maxima (log2 domain), refreshed lazily
       float l_runA = 0.f, l_runB = 0.f;           // this lane's share of the row sums
       uint32_t cur[32];        // this CTA's fp32 partial scores of the current tile
@@ -979,13 +997,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
       // completed (this warp loaded its scores) -- so that item's first Q.C^T
       // runs during this epilogue.
       have_q = false;
-      if (w + n_pairs < n_items) {
-        if (!wwait(&bar->meta_full[(k + 1) & 1], ((k + 1) >> 1) & 1, false, 336, k + 1)) {
-          ok = false;
-          break;
-        }
-      }
-      if (w + n_pairs < n_items && meta[(k + 1) & 1].has_q) {
+      if (w + n_pairs < n_items && item_has_q(p, w + n_pairs)) {
         if (!convert_q(ring, k + 1)) {
           ok = false;
           break;
