@@ -858,6 +858,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
           ok = false;
           break;
         }
+        // ... and release the S buffer as soon as the load has completed: the
+        // MMA warp's Q.C^T of tile i+2 waits for it (releasing it after this
+        // tile's maxima, to hide the load's latency, held that Q.C^T back by
+        // ~1K cycles per tile)
+        if (more) load_s_finish();
         // 2. the peer's partial scores of tile i (this warp's own barrier)
         if (lane == 0) mbar_arrive_expect_tx(&bar->x_full[sw], XBLK);
         if (!wwait(&bar->x_full[sw], gt & 1, true, 332, gt)) {
@@ -928,9 +933,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         }
         const float refA = m_runA == NEG_INF ? 0.f : m_runA;
         const float refB = m_runB == NEG_INF ? 0.f : m_runB;
-        // next tile's partial scores: wait for the TMEM load, ship
+        // next tile's partial scores to the peer
         if (more) {
-          load_s_finish();
           if (!send(gt + 1, snext)) {
             ok = false;
             break;
