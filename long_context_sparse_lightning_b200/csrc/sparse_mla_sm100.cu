@@ -239,16 +239,25 @@ __device__ __forceinline__ MlaItem mla_item_base(const MlaParams& p, int w) {
 }
 
 // The row's sequence and its descriptors (dependent loads).
+// Called by whole warps (every lane gets the same result).
 __device__ __forceinline__ void mla_item_seq(const MlaParams& p, MlaItem& it) {
-  // the row's sequence: the last b with cu_q[b] <= row (empty sequences skipped)
+  // The row's sequence: the last b with cu_q[b] <= row (empty sequences
+  // skipped).  The 32 lanes sample the remaining range at once and a ballot
+  // narrows it, so one round of loads covers 32 sequences and two cover 1024
+  // (a binary search took one dependent load per halving: ~7 cold loads for
+  // a 64-sequence decode batch).  An unsorted cu_q still yields some b in
+  // range, which the check below rejects.
+  const uint32_t lane = threadIdx.x & 31u;
   int lo = 0, hi = p.num_seqs - 1;
   while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(&p.cu_q[mid]) <= it.row) {
-      lo = mid;
-    } else {
-      hi = mid - 1;
-    }
+    const int step = (hi - lo + 32) / 32;   // ceil((hi - lo + 1) / 32)
+    const int idx = lo + static_cast<int>(lane) * step;
+    const bool le = idx <= hi && __ldg(&p.cu_q[idx]) <= it.row;
+    const uint32_t m = __ballot_sync(0xffffffffu, le);
+    if (m == 0u) break;                     // cu_q[lo] > row: no sequence holds the row
+    const int L = 31 - __clz(static_cast<int>(m));
+    lo += L * step;
+    hi = min(hi, lo + step - 1);
   }
   it.b = lo;
   const int q0 = __ldg(&p.cu_q[lo]);
