@@ -130,46 +130,43 @@ __device__ __forceinline__ float min_nan(float a, float b) {
 // Abramowitz & Stegun).  Positions below lo cost no atomic and no ranking.  The
 // fit only has to be roughly right: when fewer than k positions reach lo, the
 // histogram is rebuilt over the full range.
-template <int BLOCK, int EPT, int CAPW, typename Get4>
-__device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& get4, int n, int n_chunks, int k,
-                                            float x0, int32_t* __restrict__ out) {
-  constexpr int NW = BLOCK / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t FULL = 0xffffffffu;
-  auto pos_of = [&](int v, int c) { return (v * BLOCK + tid) * 4 + c; };
-
-  // ---- range (NaN-propagating, so any NaN or inf shows); mean and spread
-  // about x0 from a sample: the first chunk and the middle one ----
-  const int v_mid = n_chunks / 2;
-  float mx = -FLT_MAX, mn = FLT_MAX, s1 = 0.f, s2 = 0.f;
-  for_range<EPT>(0, n_chunks, [&](int v) {
-    const float4 f = get4(v);
-    const float e[4] = {f.x, f.y, f.z, f.w};
-    const bool sample = v == 0 || v == v_mid;
+// Range statistics of chunk v (4 positions from pos0): NaN-propagating max
+// and min (so any NaN or inf shows) and, for the sample chunks, the sum and
+// sum of squares about x0.  One order of operations for every caller.
+__device__ __forceinline__ void range_chunk(const float4 f, int pos0, int n, bool sample, float x0, float& mx,
+                                            float& mn, float& s1, float& s2) {
+  const float e[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (pos_of(v, c) < n) {
-        mx = max_nan(mx, e[c]);
-        mn = min_nan(mn, e[c]);
-        if (sample) {
-          const float d = e[c] - x0;
-          s1 += d;
-          s2 = fmaf(d, d, s2);
-        }
+  for (int c = 0; c < 4; ++c) {
+    if (pos0 + c < n) {
+      mx = max_nan(mx, e[c]);
+      mn = min_nan(mn, e[c]);
+      if (sample) {
+        const float d = e[c] - x0;
+        s1 += d;
+        s2 = fmaf(d, d, s2);
       }
     }
-  });
-  // butterfly reductions leave the same value in every lane (fp add commutes)
-  auto warp_all = [&](float& a, float& b, float& c, float& d) {
+  }
+}
+
+// butterfly reductions leave the same value in every lane (fp add commutes)
+__device__ __forceinline__ void range_warp_all(float& a, float& b, float& c, float& d) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      a = max_nan(a, __shfl_xor_sync(FULL, a, o));
-      b = min_nan(b, __shfl_xor_sync(FULL, b, o));
-      c += __shfl_xor_sync(FULL, c, o);
-      d += __shfl_xor_sync(FULL, d, o);
-    }
-  };
-  warp_all(mx, mn, s1, s2);
+  for (int o = 16; o > 0; o >>= 1) {
+    a = max_nan(a, __shfl_xor_sync(0xffffffffu, a, o));
+    b = min_nan(b, __shfl_xor_sync(0xffffffffu, b, o));
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    d += __shfl_xor_sync(0xffffffffu, d, o);
+  }
+}
+
+// The warp's range partials to shared memory, the histogram cleared: what
+// the range pass leaves for the block-wide reduction after a barrier.
+template <int BLOCK, int CAPW>
+__device__ __forceinline__ void range_publish(TopkShared<BLOCK, CAPW>& sh, float mx, float mn, float s1, float s2) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  range_warp_all(mx, mn, s1, s2);
   if (lane == 0) {
     sh.s_red[0][warp] = mx;
     sh.s_red[1][warp] = mn;
@@ -178,7 +175,29 @@ __device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& 
   }
   for (int j = tid; j < kBins; j += BLOCK) sh.hist[j] = 0u;
   if (tid == 0) sh.s_ncand = 0u;
-  __syncthreads();
+}
+
+// published: the caller already ran the range pass over the row (range_chunk
+// per chunk in ascending order, then range_publish) and a block barrier.
+template <int BLOCK, int EPT, int CAPW, typename Get4>
+__device__ __forceinline__ bool select_fast(TopkShared<BLOCK, CAPW>& sh, Get4&& get4, int n, int n_chunks, int k,
+                                            float x0, int32_t* __restrict__ out, bool published = false) {
+  constexpr int NW = BLOCK / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t FULL = 0xffffffffu;
+  auto pos_of = [&](int v, int c) { return (v * BLOCK + tid) * 4 + c; };
+
+  // ---- range; mean and spread about x0 from a sample: the first chunk and
+  // the middle one ----
+  const int v_mid = n_chunks / 2;
+  float mx = -FLT_MAX, mn = FLT_MAX, s1 = 0.f, s2 = 0.f;
+  if (!published) {
+    for_range<EPT>(0, n_chunks,
+                   [&](int v) { range_chunk(get4(v), pos_of(v, 0), n, v == 0 || v == v_mid, x0, mx, mn, s1, s2); });
+    range_publish(sh, mx, mn, s1, s2);
+    __syncthreads();
+  }
+  auto warp_all = [&](float& a, float& b, float& c, float& d) { range_warp_all(a, b, c, d); };
   mx = lane < NW ? sh.s_red[0][lane] : -FLT_MAX;
   mn = lane < NW ? sh.s_red[1][lane] : FLT_MAX;
   s1 = lane < NW ? sh.s_red[2][lane] : 0.f;
@@ -658,6 +677,11 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
     const int n_chunks = (n_vec + BLOCK - 1) / BLOCK;
     float x[EPT];
     const float4* b4 = reinterpret_cast<const float4*>(buf);
+    const float x0 = buf[0];
+    // the row into registers, its range pass on the way (one barrier fewer
+    // than a separate pass: the partials go out before the buffer barrier)
+    const int v_mid = n_chunks / 2;
+    float mx = -FLT_MAX, mn = FLT_MAX, s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int v = 0; v < EPT / 4; ++v) {
       const float4 f = load_padded(b4, v * BLOCK + tid, n_vec, n, false);
@@ -665,8 +689,9 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
       x[4 * v + 1] = f.y;
       x[4 * v + 2] = f.z;
       x[4 * v + 3] = f.w;
+      if (v < n_chunks) range_chunk(f, (v * BLOCK + tid) * 4, n, v == 0 || v == v_mid, x0, mx, mn, s1, s2);
     }
-    const float x0 = buf[0];
+    range_publish(sh, mx, mn, s1, s2);
     __syncthreads();   // the buffer is free: start the next row's copy
     {
       int nn;
@@ -676,7 +701,7 @@ __global__ void __launch_bounds__(BLOCK, MIN_CTAS) topk_reg_kernel(const TopkPar
       }
     }
     auto get4 = [&](int v) { return make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]); };
-    if (!select_fast<BLOCK, EPT>(sh, get4, n, n_chunks, k, x0, out)) {
+    if (!select_fast<BLOCK, EPT>(sh, get4, n, n_chunks, k, x0, out, true)) {
       const GlobalRow<BLOCK> g{reinterpret_cast<const float4*>(scores + static_cast<int64_t>(r) * p.ld), n_vec};
       select_radix<BLOCK>(sh, g, n, n_chunks, k, out);
     }
