@@ -212,7 +212,7 @@ DSA_API dsa_status_t dsa_topk_merge(int32_t n_rows, int32_t n_src, int32_t k_sel
  * the cache (q_len > kv_len, kv_start + kv_len > total_keys) records
  * DSA_ERR_DEVICE_BOUNDS and leaves that sequence's rows at out = 0, lse = -inf;
  * a row of q that lies in no sequence of cu_q (cu_q not covering 0..total_q)
- * records DSA_ERR_DEVICE_BOUNDS and is not written. */
+ * records DSA_ERR_DEVICE_BOUNDS and gets out = 0, lse = -inf as well. */
 DSA_API dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* q, int32_t n_heads, const void* kv,
                             const int32_t* idx, int32_t k_sel, float sm_scale, void* out, float* lse, void* ws,
                             size_t ws_bytes, dsa_stream_t stream);

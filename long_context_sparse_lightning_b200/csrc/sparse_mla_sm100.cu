@@ -206,7 +206,7 @@ static_assert(16 + 2 * sizeof(ItemMeta) <= 64, "item metadata fits the misc area
 // Work item w of a launch: token row w / nsplit of the batch, split w % nsplit.
 // status 0: valid; 301: the sequence's descriptors are out of range (the row
 // attends to nothing: out = 0, lse = -inf); 302: the row lies in no sequence
-// of cu_q (nothing of it is written).
+// of cu_q (the same: out = 0, lse = -inf).  Both record DSA_ERR_DEVICE_BOUNDS.
 struct MlaItem {
   int row, split, b, kv, status;
   int e_begin, e_count;   // the split's slots of the selection
@@ -1018,9 +1018,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         have_q = true;
       }
 
-      // ---- epilogue: O / l -> bf16 (or fp32 partial); nothing for a row that
-      // lies in no sequence ----
-      if (it.status != 302) {
+      // ---- epilogue: O / l -> bf16 (or fp32 partial).  An item without
+      // tiles -- a row whose selection holds no usable entry, or whose
+      // sequence is invalid (301) or absent (302) -- writes out = 0, lse =
+      // -inf (split partials: lse = -inf, which the merge turns into the
+      // same), so no stale partial of an earlier call is ever merged ----
+      {
         if (n_tiles > 0 && !wwait(&bar->pv_done, (G + n_tiles - 1) & 1, false, 335, G + n_tiles)) {
           ok = false;
           break;

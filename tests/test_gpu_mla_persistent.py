@@ -100,3 +100,40 @@ def test_forward_capped_matches_uncapped(monkeypatch):
     assert torch.equal(idx0, idx1)
     assert torch.equal(out0.view(torch.int16), out1.view(torch.int16))
     assert torch.equal(lse0, lse1)
+
+
+# (name, kv_lens, q_lens, k_sel): the bf16-cache kernel unsplit, the same split
+# (one-token rows), and the fp16-copy kernel of a prefill-shaped batch
+GAP_SHAPES = {
+    "unsplit": ([3000, 2000], [5, 4], 256),
+    "split": ([4000, 3100, 5000, 2600], [1, 1, 1, 1], 2048),
+    "fp16_copy": ([2048], [192], 512),
+}
+
+
+@pytest.mark.parametrize("shape", list(GAP_SHAPES))
+def test_row_outside_every_sequence(shape, monkeypatch):
+    # cu_q stops one row short of total_q: that row lies in no sequence.  The
+    # kernel records DSA_ERR_DEVICE_BOUNDS and gives the row out = 0 and
+    # lse = -inf (split partials: lse = -inf, so the merge cannot pick up a
+    # stale partial); every other row is computed as usual.
+    monkeypatch.delenv("DSA_MLA_MAX_PAIRS", raising=False)
+    kv, q, k_sel = GAP_SHAPES[shape]
+    x = make_inputs(custom_workload(f"persist_gap_{shape}", kv, q, k_sel=k_sel, n_heads=128), seed=63)
+    g = GpuRun(x)
+    idx = _oracle_idx(x)
+    n, H = x.batch.total_q, x.n_heads
+    g.t["cu_q"][-1] -= 1
+    out = torch.full((n, H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((n, H), float("nan"), dtype=torch.float32, device="cuda")
+    ws = dsa.workspace(dsa.OP_SPARSE_MLA, g.batch, k_sel, H)
+    ws.zero_()
+    dsa.sparse_mla(g.batch, g.t["q_mla"], g.t["latent"], torch.from_numpy(idx).cuda(), k_sel, x.sm_scale, out,
+                   lse, ws)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.check_device_error(ws)
+    assert e.value.status == 6
+    oh, lh = _host(out), _host(lse)
+    assert np.all(oh[n - 1] == 0.0) and np.all(np.isneginf(lh[n - 1]))
+    rows = list(range(n - 1))
+    check_mla(x, oh[: n - 1], lh[: n - 1], idx[: n - 1], rows)
